@@ -1,0 +1,166 @@
+/*
+ * moe.h - C ABI of the sparse-expert MoE FFN decode layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer is the one of "Uncovering Intra-expert Activation Sparsity for Efficient
+ * Mixture-of-Expert Model Execution" (technical summary, Methodology): the router picks the
+ * top-k experts of each token; every routed and every always-on shared expert computes its
+ * gate projection densely, which scores its neurons; inside each (token, expert) pair only the
+ * neurons that survive the sparsity cut are kept, and the up and down projections read and
+ * compute those neurons only; the expert outputs are combined with the routing weights.
+ *
+ * Conventions shared by every entry point
+ *   - Plain C types only.  `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Device pointers are CUDA global-memory addresses of the current device.
+ *   - The caller owns every buffer it passes.  The handle owns its workspace (allocated once
+ *     by moe_create, sized for cfg.max_tokens) and never allocates afterwards, so moe_forward
+ *     makes no allocation and no host synchronisation and may be captured in a CUDA graph.
+ *   - Element type: every x, router, weight and out buffer holds cfg.dtype (bf16 or binary32),
+ *     row-major and contiguous, 16-byte aligned.
+ *   - Errors are status codes; nothing is thrown across the ABI.  Arguments are validated
+ *     before any launch.  Faults the kernels detect (NaN router logits or activations) set an
+ *     error word on the device that moe_get_error reads.
+ *   - A handle serves one stream at a time: calls that overlap on the GPU race on its
+ *     workspace.
+ */
+#ifndef SPARSE_MOE_H_
+#define SPARSE_MOE_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* a null pointer, a size out of range, a misaligned buffer */
+  MOE_ERR_UNSUPPORTED = 2, /* a shape outside the supported limits (see moe_config) */
+  MOE_ERR_OOM = 3,         /* the workspace allocation failed */
+  MOE_ERR_CUDA = 4,        /* a CUDA call or launch failed */
+  MOE_ERR_DEVICE = 5,      /* the kernels set the device error word (moe_get_error) */
+  MOE_ERR_TIMEOUT = 6      /* reserved for bounded waits; no entry point returns it yet */
+} moe_status;
+
+typedef enum { MOE_BF16 = 0, MOE_F32 = 1 } moe_dtype;
+
+/* Routing weight of a chosen expert (the weight scales that expert's output):
+ *   SOFTMAX_TOPK  softmax over the k chosen logits
+ *   SOFTMAX_ALL   softmax over all E logits, evaluated at the chosen ones
+ *   SIGMOID       1 / (1 + exp(-logit)) of the chosen logit
+ * In every mode the k experts with the largest logits are chosen; equal logits keep the
+ * lower expert index. */
+typedef enum {
+  MOE_ROUTE_SOFTMAX_TOPK = 0,
+  MOE_ROUTE_SOFTMAX_ALL = 1,
+  MOE_ROUTE_SIGMOID = 2
+} moe_route;
+
+/* Neuron selection inside each (token, expert) pair, on the score |SiLU(g_n)|:
+ *   TOPK       keep K = I - floor(s*I + 1e-9) neurons (= ceil((1-s) I)), the largest scores;
+ *              equal scores keep the lower neuron index
+ *   THRESHOLD  keep the neurons whose score is strictly greater than `threshold` */
+typedef enum { MOE_SEL_TOPK = 0, MOE_SEL_THRESHOLD = 1 } moe_sel;
+
+/* Layer shape.  Limits: hidden in [64, 8192] and a multiple of 64; inter and inter_shared in
+ * [32, 16384] and multiples of 32; 1 <= top_k <= min(16, n_routed); n_routed <= 512;
+ * 0 <= n_shared <= 8; 1 <= max_tokens <= 1024. */
+typedef struct {
+  int hidden;       /* H */
+  int n_routed;     /* E routed experts */
+  int top_k;        /* k experts per token */
+  int inter;        /* I, intermediate size of a routed expert */
+  int n_shared;     /* S always-on shared experts (weight 1) */
+  int inter_shared; /* Ish, intermediate size of a shared expert (ignored when S = 0) */
+  int max_tokens;   /* largest n_tokens any call will pass */
+  moe_dtype dtype;
+  moe_route route;
+} moe_config;
+
+/* Selection rule for one group of experts (routed, or shared).  sparsity in [0, 1] is used in
+ * TOPK mode; threshold (binary32, may be -inf or +inf) in THRESHOLD mode. */
+typedef struct {
+  moe_sel mode;
+  double sparsity;
+  float threshold;
+} moe_sparsity;
+
+/* Packed, neuron-major expert weights (device pointers, produced by moe_pack_experts):
+ *   gate    [n][I][H]      row n = the gate weights of neuron n
+ *   updown  [n][I][2][H]   for neuron n: its W_up row, then its W_down column, contiguous,
+ *                          so a skipped neuron is 2*H*elt skipped bytes */
+typedef struct {
+  const void* gate;
+  const void* updown;
+} moe_expert_weights;
+
+typedef struct moe_handle moe_handle;
+
+/* Validates cfg, allocates the workspace for cfg->max_tokens on the current device and returns
+ * a handle in *out.  INVALID_ARG / UNSUPPORTED for a bad config, OOM if the allocation fails. */
+moe_status moe_create(const moe_config* cfg, moe_handle** out);
+
+/* Bytes of one expert's packed gate block (I*H*elt) and up/down block (2*I*H*elt); shared = 1
+ * gives the shared-expert sizes.  Either output may be NULL. */
+moe_status moe_packed_bytes(const moe_config* cfg, int shared, size_t* gate_bytes,
+                            size_t* updown_bytes);
+
+/* Re-lays n experts' logical weights into the packed layout, asynchronously on `stream`.
+ *   w_gate [n][I][H], w_up [n][I][H], w_down [n][H][I]   (device, cfg.dtype; I = Ish if shared)
+ *   packed_gate [n][I][H], packed_updown [n][I][2][H]    (device, caller-allocated)
+ * Input and output buffers must not overlap, except packed_gate == w_gate (then no copy). */
+moe_status moe_pack_experts(moe_handle* h, int shared, const void* w_gate, const void* w_up,
+                            const void* w_down, int n, void* packed_gate, void* packed_updown,
+                            void* stream);
+
+/* The layer for n_tokens tokens, asynchronously on `stream`.
+ *   x       [n_tokens][H]      device
+ *   router  [E][H]             device
+ *   routed  packed weights of the E routed experts
+ *   shared  packed weights of the S shared experts (NULL allowed when S = 0)
+ *   sp_routed, sp_shared  selection rules (sp_shared may be NULL when S = 0)
+ *   out     [n_tokens][H]      device, written
+ * n_tokens = 0 returns MOE_OK, reads no other argument and launches nothing; n_tokens < 0 or
+ * n_tokens > max_tokens is INVALID_ARG. */
+moe_status moe_forward(moe_handle* h, const void* x, int n_tokens, const void* router,
+                       const moe_expert_weights* routed, const moe_expert_weights* shared,
+                       const moe_sparsity* sp_routed, const moe_sparsity* sp_shared, void* out,
+                       void* stream);
+
+/* moe_forward with x and out in HOST memory: copies x to the handle's device staging buffer,
+ * runs the layer and copies the result back, all asynchronously on `stream` (page-locked host
+ * buffers make the copies asynchronous; the caller synchronises the stream before reading
+ * out).  Weights and router stay device pointers. */
+moe_status moe_forward_host(moe_handle* h, const void* x_host, int n_tokens, const void* router,
+                            const moe_expert_weights* routed, const moe_expert_weights* shared,
+                            const moe_sparsity* sp_routed, const moe_sparsity* sp_shared,
+                            void* out_host, void* stream);
+
+/* Copies the intermediate results of the last moe_forward (for parity checks), asynchronously
+ * on `stream`, into caller-allocated device buffers; any output may be NULL.  n_tokens must be
+ * the n_tokens of that call.  P = k + S pairs per token: pair j < k is the token's j-th routed
+ * expert (in idx order), pair k + s is shared expert s; Imax = max(I, Ish).
+ *   idx    [n_tokens][k] int32  chosen experts, by (logit desc, index asc)
+ *   w      [n_tokens][k] float  routing weights
+ *   logits [n_tokens][E] float  router logits
+ *   cnt    [n_tokens][P] int32  kept-neuron count of each pair
+ *   lists  [n_tokens][P][Imax] int32  kept neurons in ascending order, then -1 padding
+ *   act    [n_tokens][P][Imax] float  SiLU(g) of every neuron (before selection), 0 padding */
+moe_status moe_debug_lists(moe_handle* h, int n_tokens, int* idx, float* w, float* logits,
+                           int* cnt, int* lists, float* act, void* stream);
+
+/* Synchronises the device, reads and clears the device error word.  Returns MOE_ERR_DEVICE
+ * (code in *device_code: 1 = NaN router logit, 2 = NaN activation) if it was set, else MOE_OK
+ * with *device_code = 0. */
+moe_status moe_get_error(moe_handle* h, int* device_code);
+
+/* Frees the workspace and the handle (synchronises the device first).  NULL is a no-op. */
+moe_status moe_destroy(moe_handle* h);
+
+/* Static description of a status code. */
+const char* moe_status_string(moe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSE_MOE_H_ */

@@ -56,6 +56,7 @@ def _bind(lib):
     lib.oracle_threads.restype = ctypes.c_int
     lib.oracle_route.argtypes = [ctypes.POINTER(_Layer), P, ctypes.c_int, P, P, P]
     lib.oracle_route_weights.argtypes = [ctypes.POINTER(_Layer), P, P, P]
+    lib.oracle_topk.argtypes = [P, ctypes.c_int, ctypes.c_int, P]
     lib.oracle_gate.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P]
     lib.oracle_select.argtypes = [P, ctypes.c_int, _Sel, P]
     lib.oracle_expert.argtypes = [P, P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P]
@@ -63,7 +64,7 @@ def _bind(lib):
                                    P, P, P, P, P, P, ctypes.c_int]
     lib.oracle_calibrate.argtypes = [ctypes.POINTER(_Layer), P, ctypes.c_int, ctypes.c_int,
                                      ctypes.c_double, P, P, ctypes.c_int]
-    for f in ("oracle_route", "oracle_route_weights", "oracle_gate", "oracle_select",
+    for f in ("oracle_route", "oracle_route_weights", "oracle_topk", "oracle_gate", "oracle_select",
               "oracle_expert", "oracle_forward", "oracle_calibrate"):
         getattr(lib, f).restype = ctypes.c_int
     return lib
@@ -116,10 +117,14 @@ class Layer:
         self._g, self._u, self._d = arr(), arr(), arr()
         self._sg, self._su, self._sd = sarr(), sarr(), sarr()
         for e, (g, u, d) in experts.items():
-            g, u, d = (np.ascontiguousarray(v) for v in (g, u, d))
-            assert g.shape == (shape.inter, shape.hidden) and d.shape == (shape.hidden, shape.inter)
-            self._keep += [g, u, d]
-            self._g[e], self._u[e], self._d[e] = g.ctypes.data, u.ctypes.data, d.ctypes.data
+            # up/down may be None when only the gate is needed (threshold calibration)
+            g, u, d = (None if v is None else np.ascontiguousarray(v) for v in (g, u, d))
+            assert g.shape == (shape.inter, shape.hidden)
+            assert d is None or d.shape == (shape.hidden, shape.inter)
+            self._keep += [v for v in (g, u, d) if v is not None]
+            self._g[e] = g.ctypes.data
+            self._u[e] = None if u is None else u.ctypes.data
+            self._d[e] = None if d is None else d.ctypes.data
         for s, (g, u, d) in enumerate(shared):
             g, u, d = (np.ascontiguousarray(v) for v in (g, u, d))
             self._keep += [g, u, d]
@@ -191,6 +196,15 @@ def keep_count(I, s, lib=None):
 
 def threads(lib=None):
     return int((lib or load()).oracle_threads())
+
+
+def topk(logits_row, k, lib=None):
+    """The k experts of one token's logits by (logit desc, index asc)."""
+    lib = lib or load()
+    lg = np.ascontiguousarray(logits_row, dtype=np.float64)
+    idx = np.zeros(k, np.int32)
+    _check(lib.oracle_topk(_ptr(lg), lg.shape[0], int(k), _ptr(idx)), "oracle_topk")
+    return idx
 
 
 def gate(x_t, wg, lib=None):

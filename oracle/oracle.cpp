@@ -235,6 +235,13 @@ int oracle_route(const oracle_layer* L, const void* x, int B, double* logits, in
   return ORACLE_OK;
 }
 
+/* The top-k experts of given logits [E] by (logit descending, index ascending). */
+int oracle_topk(const double* logits, int E, int k, int* idx) {
+  if (!logits || !idx || E <= 0 || k <= 0 || k > E) return ORACLE_BAD_ARG;
+  topk_experts(logits, E, k, idx);
+  return ORACLE_OK;
+}
+
 /* Routing weights for a given choice of experts idx[0..k) and the token's logits [E]. */
 int oracle_route_weights(const oracle_layer* L, const double* logits, const int* idx, double* w) {
   if (!L || !logits || !idx || !w) return ORACLE_BAD_ARG;

@@ -1,0 +1,187 @@
+// common.cuh - device helpers shared by the layer's kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kThreads = 256;      // threads of the gate / up-down / router CTAs
+constexpr int kWarps = kThreads / 32;
+constexpr int kTileTok = 8;        // tokens per tile (the n of an m16n8k16 mma)
+constexpr int kTileRows = 16;      // rows per tile (the m of an m16n8k16 mma)
+constexpr int kMaxTopK = 16;
+constexpr int kMaxShared = 8;
+constexpr int kMaxRouted = 512;
+constexpr int kMaxTokens = 1024;
+
+// device error word codes
+constexpr int kErrNanLogit = 1;
+constexpr int kErrNanAct = 2;
+
+// One expert that this call evaluates: a routed expert with >= 1 token, or a shared expert.
+struct Slot {
+  int kind;    // 0 routed, 1 shared
+  int expert;  // routed expert index, or shared expert index
+  int T;       // tokens of this expert
+  int q0;      // first pair index of its tokens (pairs of a slot are contiguous, tokens ascending)
+  int I;       // intermediate size
+  int item0;   // first gate work item of this slot
+  int pad0, pad1;
+};
+
+// meta words written by the router kernel
+enum { kMetaSlots = 0, kMetaPairs = 1, kMetaGateItems = 2, kMetaTouched = 3, kMetaWords = 8 };
+
+struct FwdParams {
+  int H, E, k, S, I, Ish, B, Imax;
+  int route;
+  int sel_mode[2];  // [0] routed, [1] shared: 0 top-K, 1 threshold
+  int sel_K[2];
+  float sel_t[2];
+  const void* x;
+  const void* router;
+  const void* gate_r;
+  const void* updown_r;
+  const void* gate_s;
+  const void* updown_s;
+  void* out;
+  // workspace
+  float* logits;       // [Bmax][E]
+  int* topk_idx;       // [Bmax][k]
+  float* topk_w;       // [Bmax][k]
+  int* pair_index;     // [Bmax][k+S]
+  int* pair_token;     // [Pmax]
+  float* pair_w;       // [Pmax]
+  int* pair_slot;      // [Pmax]
+  Slot* slots;         // [E+S]
+  int* meta;           // [kMetaWords]
+  unsigned* tile_ticket;   // [ceil(Bmax/8)]
+  unsigned* global_ticket; // [1]
+  unsigned* slot_ticket;   // [E+S]
+  float* act;          // [Pmax][Imax]
+  uint32_t* maskbits;  // [Pmax][Imax/32]
+  int* lists;          // [Pmax][Imax]
+  int* cnt;            // [Pmax]
+  uint32_t* ubits;     // [E+S][Imax/32]
+  int* ulist;          // [E+S][Imax]
+  int* ucnt;           // [E+S]
+  float* out_acc;      // [Bmax][H]
+  int* err;            // device error word
+};
+
+// ---------------------------------------------------------------------------------------------
+// Programmatic dependent launch: a kernel launched with the programmatic-serialization attribute
+// may start while its predecessor runs; it must wait before it reads the predecessor's output.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------------------------
+// loads
+__device__ __forceinline__ uint4 ld_stream(const void* p) {  // read-once weights: skip L1
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint4 ld_nc(const void* p) {  // read-only, reused: through L1
+  return __ldg(reinterpret_cast<const uint4*>(p));
+}
+__device__ __forceinline__ int ld_cg(const int* p) { return __ldcg(p); }
+__device__ __forceinline__ unsigned ld_cg(const unsigned* p) { return __ldcg(p); }
+__device__ __forceinline__ float ld_cg(const float* p) { return __ldcg(p); }
+
+// fp32 vector reduction into global memory (sm_90+)
+__device__ __forceinline__ void red_add_v2(float* p, float a, float b) {
+  asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(a), "f"(b) : "memory");
+}
+
+// ---------------------------------------------------------------------------------------------
+// bf16 helpers
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// D += A * B, m16n8k16, bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_16816(float d[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// ---------------------------------------------------------------------------------------------
+// scans and reductions
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Exclusive prefix sum of v over the block (blockDim.x a multiple of 32, <= 1024); scratch holds
+// 33 ints.  Returns the exclusive prefix; *total gets the block sum.  Contains __syncthreads.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) scratch[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int s = lane < nw ? scratch[lane] : 0;
+    int si = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, si, o);
+      if (lane >= o) si += y;
+    }
+    if (lane < nw) scratch[lane] = si - s;
+    if (lane == 31) scratch[32] = si;
+  }
+  __syncthreads();
+  int res = scratch[warp] + incl - v;
+  if (total) *total = scratch[32];
+  __syncthreads();
+  return res;
+}
+
+__device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
+
+__device__ __forceinline__ void set_error(int* err, int code) { atomicCAS(err, 0, code); }
+
+template <typename T>
+struct Elt;
+template <>
+struct Elt<__nv_bfloat16> {
+  static constexpr int kBytes = 2;
+  static constexpr int kPerVec = 8;  // elements per 16-byte vector
+};
+template <>
+struct Elt<float> {
+  static constexpr int kBytes = 4;
+  static constexpr int kPerVec = 4;
+};
+
+// Slot lookup: index j with items[j] <= i < items[j+1] (items ascending, n entries + sentinel).
+__device__ __forceinline__ int find_slot(const int* items, int n, int i) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (items[mid] <= i) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+}  // namespace moe

@@ -1,0 +1,53 @@
+// kernels.h - host-side launchers of the layer's kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+struct LaunchShape {
+  int nsm;            // SMs of the device
+  int grid_gate;      // persistent grid of the gate kernel
+  int grid_updown;    // persistent grid of the up/down kernel
+  int grid_select;    // cap of the selection grid
+};
+
+// dtype: 0 bf16, 1 fp32.  Each launcher returns the launch's cudaError_t.
+cudaError_t launch_router(const FwdParams& p, int dtype, cudaStream_t st);
+cudaError_t launch_gate(const FwdParams& p, int dtype, const LaunchShape& ls, cudaStream_t st);
+cudaError_t launch_select(const FwdParams& p, const LaunchShape& ls, cudaStream_t st);
+cudaError_t launch_updown(const FwdParams& p, int dtype, const LaunchShape& ls, cudaStream_t st);
+cudaError_t launch_finalize(const FwdParams& p, int dtype, const LaunchShape& ls, cudaStream_t st);
+
+// Set-up (called once per handle): shared-memory limits and persistent grid sizes.
+cudaError_t configure_kernels(int dtype, int imax, int max_E, int max_B, LaunchShape* ls);
+size_t router_smem_bytes(int E, int B);
+size_t select_smem_bytes(int imax);
+
+// Packing and debug export.
+cudaError_t launch_pack_down(const void* w_down, void* packed_updown, int n, int I, int H,
+                             int elt, cudaStream_t st);
+cudaError_t launch_debug_gather(const FwdParams& p, int n_tokens, int* cnt, int* lists,
+                                float* act, cudaStream_t st);
+
+// cudaLaunchKernelEx with programmatic stream serialization (the kernel may start while its
+// predecessor in the stream runs and calls griddepcontrol.wait before reading its results).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, bool pdl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+}  // namespace moe

@@ -1,0 +1,120 @@
+// misc.cu - output cast, weight packing, debug export and per-handle kernel configuration.
+#include "kernels.h"
+
+namespace moe {
+
+int gate_occupancy(int dtype);
+int updown_occupancy(int dtype);
+cudaError_t configure_router(int max_E, int max_B);
+cudaError_t configure_select(int imax, int* occupancy);
+
+namespace {
+
+// out[t][h] = dtype(out_acc[t][h]); out_acc is cleared for the next call.
+template <typename T>
+__global__ void finalize_kernel(FwdParams p) {
+  pdl_trigger();
+  pdl_wait();
+  const size_t n4 = (size_t)p.B * p.H / 4;
+  float4* acc = reinterpret_cast<float4*>(p.out_acc);
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const float4 v = __ldcg(acc + i);
+    acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if constexpr (sizeof(T) == 2) {
+      uint2 o;
+      o.x = pack_bf16x2(v.x, v.y);
+      o.y = pack_bf16x2(v.z, v.w);
+      reinterpret_cast<uint2*>(p.out)[i] = o;
+    } else {
+      reinterpret_cast<float4*>(p.out)[i] = v;
+    }
+  }
+}
+
+// packed[e][n][1][h] = w_down[e][h][n]: 32x32 tiles through shared memory.
+template <typename T>
+__global__ void pack_down_kernel(const T* __restrict__ wd, T* __restrict__ ud, int I, int H) {
+  __shared__ T tile[32][33];
+  const int e = blockIdx.z;
+  const int n0 = blockIdx.x * 32, h0 = blockIdx.y * 32;
+  const T* src = wd + (size_t)e * H * I;
+  T* dst = ud + (size_t)e * I * 2 * H;
+  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+    const int h = h0 + r, n = n0 + threadIdx.x;
+    if (h < H && n < I) tile[r][threadIdx.x] = src[(size_t)h * I + n];
+  }
+  __syncthreads();
+  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+    const int n = n0 + r, h = h0 + threadIdx.x;
+    if (h < H && n < I) dst[(size_t)n * 2 * H + H + h] = tile[threadIdx.x][r];
+  }
+}
+
+// Reorders the per-pair lists / counts / activations of the last call into [token][pair] order.
+__global__ void debug_gather_kernel(FwdParams p, int* cnt, int* lists, float* act) {
+  const int P = p.k + p.S;
+  const int tj = blockIdx.x;  // token * P + pair
+  const int t = tj / P, jj = tj % P;
+  const int q = p.pair_index[t * P + jj];
+  const int I = jj < p.k ? p.I : p.Ish;
+  const int c = p.cnt[q];
+  if (threadIdx.x == 0 && cnt) cnt[tj] = c;
+  for (int n = threadIdx.x; n < p.Imax; n += blockDim.x) {
+    if (lists) lists[(size_t)tj * p.Imax + n] = n < c ? p.lists[(size_t)q * p.Imax + n] : -1;
+    if (act) act[(size_t)tj * p.Imax + n] = n < I ? p.act[(size_t)q * p.Imax + n] : 0.f;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_finalize(const FwdParams& p, int dtype, const LaunchShape& ls, cudaStream_t st) {
+  const size_t n4 = (size_t)p.B * p.H / 4;
+  size_t blocks = (n4 + 255) / 256;
+  const size_t cap = (size_t)ls.nsm * 4;
+  if (blocks > cap) blocks = cap;
+  if (dtype == 0)
+    return launch_pdl(finalize_kernel<__nv_bfloat16>, dim3((unsigned)blocks), dim3(256), 0, st,
+                      true, p);
+  return launch_pdl(finalize_kernel<float>, dim3((unsigned)blocks), dim3(256), 0, st, true, p);
+}
+
+cudaError_t launch_pack_down(const void* w_down, void* packed_updown, int n, int I, int H,
+                             int elt, cudaStream_t st) {
+  dim3 grid((I + 31) / 32, (H + 31) / 32, n), block(32, 8);
+  if (elt == 2)
+    pack_down_kernel<__nv_bfloat16><<<grid, block, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(w_down), static_cast<__nv_bfloat16*>(packed_updown), I, H);
+  else
+    pack_down_kernel<float><<<grid, block, 0, st>>>(static_cast<const float*>(w_down),
+                                                    static_cast<float*>(packed_updown), I, H);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_debug_gather(const FwdParams& p, int n_tokens, int* cnt, int* lists,
+                                float* act, cudaStream_t st) {
+  const int P = p.k + p.S;
+  debug_gather_kernel<<<n_tokens * P, 256, 0, st>>>(p, cnt, lists, act);
+  return cudaGetLastError();
+}
+
+cudaError_t configure_kernels(int dtype, int imax, int max_E, int max_B, LaunchShape* ls) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&ls->nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  e = configure_router(max_E, max_B);
+  if (e != cudaSuccess) return e;
+  int occ_sel = 0;
+  e = configure_select(imax, &occ_sel);
+  if (e != cudaSuccess) return e;
+  const int occ_gate = gate_occupancy(dtype);
+  const int occ_ud = updown_occupancy(dtype);
+  ls->grid_gate = ls->nsm * (occ_gate > 0 ? occ_gate : 1);
+  ls->grid_updown = ls->nsm * (occ_ud > 0 ? occ_ud : 1);
+  ls->grid_select = ls->nsm * (occ_sel > 0 ? occ_sel : 1);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,372 @@
+// moe_api.cu - the C ABI declared in include/moe.h: argument checks, the workspace, packing,
+// and the launch sequence of one layer call.
+//
+// One call runs five kernels on the caller's stream, each (after the first) launched with
+// programmatic dependent launch so that it is resident before its predecessor drains:
+//   router   logits, top-k, routing weights, pair grouping and slot table
+//   gate     dense gate + SiLU of every evaluated pair
+//   select   per-pair kept set, per-expert union of kept neurons
+//   updown   sparse up/down over the kept rows, weighted into an fp32 accumulator
+//   finalize accumulator -> out (dtype), accumulator cleared
+// Nothing is allocated and nothing waits on the host, so a call can be captured in a graph.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <new>
+
+#include "../../include/moe.h"
+#include "kernels.h"
+
+using moe::FwdParams;
+using moe::LaunchShape;
+
+struct moe_handle {
+  moe_config cfg;
+  int device;
+  int elt;
+  int imax;
+  LaunchShape ls;
+  FwdParams base;  // workspace pointers and sizes
+  void* ws;
+  size_t ws_bytes;
+  void* zero_begin;  // [zero_begin, zero_begin + zero_bytes) is all-zero between calls
+  size_t zero_bytes;
+  void* x_stage;    // device staging of moe_forward_host
+  void* out_stage;
+  bool dirty;       // a call failed mid-way: re-zero before the next one
+  int last_tokens;
+};
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status check_config(const moe_config* c) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->dtype != MOE_BF16 && c->dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
+  if (c->route < MOE_ROUTE_SOFTMAX_TOPK || c->route > MOE_ROUTE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (c->hidden <= 0 || c->n_routed <= 0 || c->top_k <= 0 || c->inter <= 0 ||
+      c->max_tokens <= 0 || c->n_shared < 0 || (c->n_shared > 0 && c->inter_shared <= 0))
+    return MOE_ERR_INVALID_ARG;
+  if (c->top_k > c->n_routed) return MOE_ERR_INVALID_ARG;
+  if (c->hidden % 64 || c->hidden < 64 || c->hidden > 8192) return MOE_ERR_UNSUPPORTED;
+  if (c->inter % 32 || c->inter < 32 || c->inter > 16384) return MOE_ERR_UNSUPPORTED;
+  if (c->n_shared > 0 && (c->inter_shared % 32 || c->inter_shared < 32 || c->inter_shared > 16384))
+    return MOE_ERR_UNSUPPORTED;
+  if (c->top_k > moe::kMaxTopK || c->n_routed > moe::kMaxRouted || c->n_shared > moe::kMaxShared ||
+      c->max_tokens > moe::kMaxTokens)
+    return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status check_sparsity(const moe_sparsity* s) {
+  if (!s) return MOE_ERR_INVALID_ARG;
+  if (s->mode == MOE_SEL_TOPK) {
+    if (!(s->sparsity >= 0.0 && s->sparsity <= 1.0)) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+  }
+  if (s->mode == MOE_SEL_THRESHOLD) return isnan(s->threshold) ? MOE_ERR_INVALID_ARG : MOE_OK;
+  return MOE_ERR_INVALID_ARG;
+}
+
+// K = ceil((1 - s) I), evaluated as I - floor(s I + 1e-9) and clamped to [0, I].
+int keep_count(int I, double s) {
+  long k = (long)I - (long)floor(s * (double)I + 1e-9);
+  if (k < 0) k = 0;
+  if (k > I) k = I;
+  return (int)k;
+}
+
+struct Carve {
+  char* base;
+  size_t off;
+  template <typename T>
+  T* take(size_t n) {
+    off = (off + 255) & ~(size_t)255;
+    T* p = reinterpret_cast<T*>(base + off);
+    off += n * sizeof(T);
+    return p;
+  }
+};
+
+// Lays the workspace out (base == nullptr only measures it).
+size_t carve(moe_handle* h, char* base) {
+  const moe_config& c = h->cfg;
+  const size_t Bm = (size_t)c.max_tokens, E = c.n_routed, k = c.top_k, S = c.n_shared;
+  const size_t Pm = Bm * (k + S), Im = h->imax, Wm = Im / 32, slots = E + S;
+  Carve cv{base, 0};
+  FwdParams& p = h->base;
+  p.logits = cv.take<float>(Bm * E);
+  p.topk_idx = cv.take<int>(Bm * k);
+  p.topk_w = cv.take<float>(Bm * k);
+  p.pair_index = cv.take<int>(Bm * (k + S));
+  p.pair_token = cv.take<int>(Pm);
+  p.pair_w = cv.take<float>(Pm);
+  p.pair_slot = cv.take<int>(Pm);
+  p.slots = cv.take<moe::Slot>(slots);
+  p.meta = cv.take<int>(moe::kMetaWords);
+  p.act = cv.take<float>(Pm * Im);
+  p.maskbits = cv.take<uint32_t>(Pm * Wm);
+  p.lists = cv.take<int>(Pm * Im);
+  p.cnt = cv.take<int>(Pm);
+  p.ulist = cv.take<int>(slots * Im);
+  p.ucnt = cv.take<int>(slots);
+  p.err = cv.take<int>(1);
+  h->x_stage = cv.take<char>(Bm * c.hidden * h->elt);
+  h->out_stage = cv.take<char>(Bm * c.hidden * h->elt);
+  // zero-at-rest region: tickets, union bitmasks, output accumulator
+  char* zb = cv.take<char>(0);
+  p.tile_ticket = cv.take<unsigned>((Bm + moe::kTileTok - 1) / moe::kTileTok);
+  p.global_ticket = cv.take<unsigned>(1);
+  p.slot_ticket = cv.take<unsigned>(slots);
+  p.ubits = cv.take<uint32_t>(slots * Wm);
+  p.out_acc = cv.take<float>(Bm * c.hidden);
+  h->zero_begin = zb;
+  h->zero_bytes = (size_t)((base + cv.off) - zb);
+  return cv.off + 256;
+}
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+moe_status forward_impl(moe_handle* h, const void* x, int n_tokens, const void* router,
+                        const moe_expert_weights* routed, const moe_expert_weights* shared,
+                        const moe_sparsity* sp_routed, const moe_sparsity* sp_shared, void* out,
+                        cudaStream_t st) {
+  const moe_config& c = h->cfg;
+  FwdParams p = h->base;
+  p.H = c.hidden;
+  p.E = c.n_routed;
+  p.k = c.top_k;
+  p.S = c.n_shared;
+  p.I = c.inter;
+  p.Ish = c.n_shared > 0 ? c.inter_shared : 0;
+  p.B = n_tokens;
+  p.Imax = h->imax;
+  p.route = (int)c.route;
+  p.sel_mode[0] = sp_routed->mode == MOE_SEL_THRESHOLD ? 1 : 0;
+  p.sel_K[0] = keep_count(c.inter, sp_routed->sparsity);
+  p.sel_t[0] = sp_routed->threshold;
+  if (c.n_shared > 0) {
+    p.sel_mode[1] = sp_shared->mode == MOE_SEL_THRESHOLD ? 1 : 0;
+    p.sel_K[1] = keep_count(c.inter_shared, sp_shared->sparsity);
+    p.sel_t[1] = sp_shared->threshold;
+  } else {
+    p.sel_mode[1] = 0;
+    p.sel_K[1] = 0;
+    p.sel_t[1] = 0.f;
+  }
+  p.x = x;
+  p.router = router;
+  p.gate_r = routed->gate;
+  p.updown_r = routed->updown;
+  p.gate_s = c.n_shared > 0 ? shared->gate : nullptr;
+  p.updown_s = c.n_shared > 0 ? shared->updown : nullptr;
+  p.out = out;
+  if (h->dirty) {
+    if (cudaMemsetAsync(h->zero_begin, 0, h->zero_bytes, st) != cudaSuccess) return MOE_ERR_CUDA;
+    h->dirty = false;
+  }
+  const int dt = c.dtype == MOE_BF16 ? 0 : 1;
+  cudaError_t e = moe::launch_router(p, dt, st);
+  if (e == cudaSuccess) e = moe::launch_gate(p, dt, h->ls, st);
+  if (e == cudaSuccess) e = moe::launch_select(p, h->ls, st);
+  if (e == cudaSuccess) e = moe::launch_updown(p, dt, h->ls, st);
+  if (e == cudaSuccess) e = moe::launch_finalize(p, dt, h->ls, st);
+  if (e != cudaSuccess) {
+    h->dirty = true;
+    return MOE_ERR_CUDA;
+  }
+  h->last_tokens = n_tokens;
+  return MOE_OK;
+}
+
+moe_status check_forward(moe_handle* h, const void* x, int n_tokens, const void* router,
+                         const moe_expert_weights* routed, const moe_expert_weights* shared,
+                         const moe_sparsity* sp_routed, const moe_sparsity* sp_shared,
+                         const void* out, bool host_io) {
+  if (!h || n_tokens < 0 || n_tokens > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+  if (n_tokens == 0) return MOE_OK;  // a no-op: nothing is read
+  if (!x || !router || !routed || !out || !sp_routed) return MOE_ERR_INVALID_ARG;
+  if (!routed->gate || !routed->updown) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(router) || !aligned16(routed->gate) || !aligned16(routed->updown))
+    return MOE_ERR_INVALID_ARG;
+  if (!host_io && (!aligned16(x) || !aligned16(out))) return MOE_ERR_INVALID_ARG;
+  moe_status s = check_sparsity(sp_routed);
+  if (s != MOE_OK) return s;
+  if (h->cfg.n_shared > 0) {
+    if (!shared || !shared->gate || !shared->updown || !sp_shared) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(shared->gate) || !aligned16(shared->updown)) return MOE_ERR_INVALID_ARG;
+    s = check_sparsity(sp_shared);
+    if (s != MOE_OK) return s;
+  }
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_create(const moe_config* cfg, moe_handle** out) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  moe_handle* h = new (std::nothrow) moe_handle();
+  if (!h) return MOE_ERR_OOM;
+  h->cfg = *cfg;
+  h->elt = cfg->dtype == MOE_BF16 ? 2 : 4;
+  h->imax = cfg->inter;
+  if (cfg->n_shared > 0 && cfg->inter_shared > h->imax) h->imax = cfg->inter_shared;
+  if (cudaGetDevice(&h->device) != cudaSuccess) {
+    delete h;
+    return MOE_ERR_CUDA;
+  }
+  cudaError_t e = moe::configure_kernels(cfg->dtype == MOE_BF16 ? 0 : 1, h->imax, cfg->n_routed,
+                                         cfg->max_tokens, &h->ls);
+  if (e != cudaSuccess) {
+    delete h;
+    return MOE_ERR_CUDA;
+  }
+  h->ws_bytes = carve(h, nullptr);
+  if (cudaMalloc(&h->ws, h->ws_bytes) != cudaSuccess) {
+    cudaGetLastError();
+    delete h;
+    return MOE_ERR_OOM;
+  }
+  carve(h, static_cast<char*>(h->ws));
+  if (cudaMemset(h->ws, 0, h->ws_bytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+    cudaFree(h->ws);
+    delete h;
+    return MOE_ERR_CUDA;
+  }
+  *out = h;
+  return MOE_OK;
+}
+
+moe_status moe_packed_bytes(const moe_config* cfg, int shared, size_t* gate_bytes,
+                            size_t* updown_bytes) {
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  if (shared && cfg->n_shared == 0) return MOE_ERR_INVALID_ARG;
+  const size_t elt = cfg->dtype == MOE_BF16 ? 2 : 4;
+  const size_t I = shared ? cfg->inter_shared : cfg->inter;
+  if (gate_bytes) *gate_bytes = I * cfg->hidden * elt;
+  if (updown_bytes) *updown_bytes = 2 * I * cfg->hidden * elt;
+  return MOE_OK;
+}
+
+moe_status moe_pack_experts(moe_handle* h, int shared, const void* w_gate, const void* w_up,
+                            const void* w_down, int n, void* packed_gate, void* packed_updown,
+                            void* stream) {
+  if (!h || !w_gate || !w_up || !w_down || !packed_gate || !packed_updown || n < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (shared && h->cfg.n_shared == 0) return MOE_ERR_INVALID_ARG;
+  if (n > (shared ? h->cfg.n_shared : h->cfg.n_routed)) return MOE_ERR_INVALID_ARG;
+  if (n == 0) return MOE_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t H = h->cfg.hidden, I = shared ? h->cfg.inter_shared : h->cfg.inter, elt = h->elt;
+  cudaError_t e = cudaSuccess;
+  if (packed_gate != w_gate)
+    e = cudaMemcpyAsync(packed_gate, w_gate, (size_t)n * I * H * elt, cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess)
+    e = cudaMemcpy2DAsync(packed_updown, 2 * H * elt, w_up, H * elt, H * elt, (size_t)n * I,
+                          cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess) e = moe::launch_pack_down(w_down, packed_updown, n, (int)I, (int)H, (int)elt, st);
+  return cuda_status(e);
+}
+
+moe_status moe_forward(moe_handle* h, const void* x, int n_tokens, const void* router,
+                       const moe_expert_weights* routed, const moe_expert_weights* shared,
+                       const moe_sparsity* sp_routed, const moe_sparsity* sp_shared, void* out,
+                       void* stream) {
+  moe_status s = check_forward(h, x, n_tokens, router, routed, shared, sp_routed, sp_shared, out,
+                               false);
+  if (s != MOE_OK) return s;
+  if (n_tokens == 0) return MOE_OK;
+  return forward_impl(h, x, n_tokens, router, routed, shared, sp_routed, sp_shared, out,
+                      static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_forward_host(moe_handle* h, const void* x_host, int n_tokens, const void* router,
+                            const moe_expert_weights* routed, const moe_expert_weights* shared,
+                            const moe_sparsity* sp_routed, const moe_sparsity* sp_shared,
+                            void* out_host, void* stream) {
+  moe_status s = check_forward(h, x_host, n_tokens, router, routed, shared, sp_routed, sp_shared,
+                               out_host, true);
+  if (s != MOE_OK) return s;
+  if (n_tokens == 0) return MOE_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t bytes = (size_t)n_tokens * h->cfg.hidden * h->elt;
+  if (cudaMemcpyAsync(h->x_stage, x_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  s = forward_impl(h, h->x_stage, n_tokens, router, routed, shared, sp_routed, sp_shared,
+                   h->out_stage, st);
+  if (s != MOE_OK) return s;
+  if (cudaMemcpyAsync(out_host, h->out_stage, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status moe_debug_lists(moe_handle* h, int n_tokens, int* idx, float* w, float* logits,
+                           int* cnt, int* lists, float* act, void* stream) {
+  if (!h || n_tokens <= 0 || n_tokens != h->last_tokens) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const moe_config& c = h->cfg;
+  FwdParams p = h->base;
+  p.H = c.hidden;
+  p.E = c.n_routed;
+  p.k = c.top_k;
+  p.S = c.n_shared;
+  p.I = c.inter;
+  p.Ish = c.n_shared > 0 ? c.inter_shared : 0;
+  p.B = n_tokens;
+  p.Imax = h->imax;
+  cudaError_t e = cudaSuccess;
+  const size_t nk = (size_t)n_tokens * c.top_k;
+  if (idx) e = cudaMemcpyAsync(idx, p.topk_idx, nk * sizeof(int), cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess && w)
+    e = cudaMemcpyAsync(w, p.topk_w, nk * sizeof(float), cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess && logits)
+    e = cudaMemcpyAsync(logits, p.logits, (size_t)n_tokens * c.n_routed * sizeof(float),
+                        cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess && (cnt || lists || act))
+    e = moe::launch_debug_gather(p, n_tokens, cnt, lists, act, st);
+  return cuda_status(e);
+}
+
+moe_status moe_get_error(moe_handle* h, int* device_code) {
+  if (!h || !device_code) return MOE_ERR_INVALID_ARG;
+  *device_code = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, h->base.err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (v == 0) return MOE_OK;
+  *device_code = v;
+  if (cudaMemset(h->base.err, 0, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_ERR_DEVICE;
+}
+
+moe_status moe_destroy(moe_handle* h) {
+  if (!h) return MOE_OK;
+  cudaError_t e = cudaDeviceSynchronize();
+  cudaError_t f = cudaFree(h->ws);
+  delete h;
+  return (e == cudaSuccess && f == cudaSuccess) ? MOE_OK : MOE_ERR_CUDA;
+}
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape";
+    case MOE_ERR_OOM: return "out of device memory";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE: return "device-side error flag set";
+    case MOE_ERR_TIMEOUT: return "timeout";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

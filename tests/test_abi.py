@@ -1,0 +1,93 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point that include/moe.h
+declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_expert_ffn_logits_b200 as moe
+from sparse_expert_ffn_logits_b200 import build as moe_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    moe_build.build()
+    return moe.load()
+
+
+def declared_entry_points():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:moe_status|size_t|const char\s*\*)\s*(moe_\w+)\s*\(",
+                                 src, flags=re.M)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_entry_points()
+    assert len(names) >= 9, names
+    for n in names:
+        assert hasattr(lib, n), f"{n} not exported"
+    assert set(names) == set(moe.EXPORTS)
+
+
+def _cfg(**kw):
+    base = dict(hidden=2048, n_routed=64, top_k=8, inter=1024, n_shared=0, inter_shared=0,
+                max_tokens=16, dtype="bf16", route="softmax_topk")
+    base.update(kw)
+    return moe.make_config(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(hidden=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(top_k=65), moe.MOE_ERR_INVALID_ARG),
+    (dict(max_tokens=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(n_shared=1, inter_shared=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(dtype=7), moe.MOE_ERR_INVALID_ARG),
+    (dict(route=9), moe.MOE_ERR_INVALID_ARG),
+    (dict(hidden=2000), moe.MOE_ERR_UNSUPPORTED),
+    (dict(hidden=16384), moe.MOE_ERR_UNSUPPORTED),
+    (dict(inter=1000), moe.MOE_ERR_UNSUPPORTED),
+    (dict(top_k=17, n_routed=64), moe.MOE_ERR_UNSUPPORTED),
+    (dict(n_routed=1024, top_k=2), moe.MOE_ERR_UNSUPPORTED),
+    (dict(max_tokens=4096), moe.MOE_ERR_UNSUPPORTED),
+    (dict(n_shared=9, inter_shared=1024), moe.MOE_ERR_UNSUPPORTED),
+])
+def test_create_rejects_bad_config(lib, kw, status):
+    h = ctypes.c_void_p()
+    assert lib.moe_create(ctypes.byref(_cfg(**kw)), ctypes.byref(h)) == status
+    assert not h.value
+
+
+def test_create_null_args(lib):
+    h = ctypes.c_void_p()
+    assert lib.moe_create(None, ctypes.byref(h)) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_create(ctypes.byref(_cfg()), None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_packed_bytes(lib):
+    assert moe.moe_packed_bytes(_cfg()) == (1024 * 2048 * 2, 2 * 1024 * 2048 * 2)
+    c = _cfg(dtype="f32", n_shared=2, inter_shared=1408)
+    assert moe.moe_packed_bytes(c, shared=1) == (1408 * 2048 * 4, 2 * 1408 * 2048 * 4)
+    with pytest.raises(moe.MoEError):
+        moe.moe_packed_bytes(_cfg(), shared=1)
+
+
+def test_forward_rejects_null_handle(lib):
+    rw = moe.MoEExpertWeights(16, 16)
+    sp = moe.sparsity(("topk", 0.5))
+    rc = lib.moe_forward(None, ctypes.c_void_p(16), 1, ctypes.c_void_p(16), ctypes.byref(rw), None,
+                         ctypes.byref(sp), None, ctypes.c_void_p(16), None)
+    assert rc == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_get_error(None, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_destroy(None) == moe.MOE_OK
+    assert lib.moe_debug_lists(None, 1, None, None, None, None, None, None, None) == \
+        moe.MOE_ERR_INVALID_ARG
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert lib.moe_status_string(s)
+    assert lib.moe_status_string(99) == b"unknown status"

@@ -1,0 +1,205 @@
+"""CUDA layer vs the fp64 oracle on the five workloads, through the C ABI (see parity.py for
+the comparison rules).  Every input is drawn by the seeded generator; the device copy is drawn
+on the GPU and the oracle's copy on the host, and the two are checked to be the same bits."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from sparse_expert_ffn_logits_b200 import (MOE_ERR_DEVICE, MOE_OK, moe_get_error)
+from sparse_expert_ffn_logits_b200.workload import DeviceLayer
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+def _tokens(dl, B, batch_index):
+    seed = synth.token_seed(dl.shape, batch_index)
+    return synth.host_tokens(dl.shape, B, seed), dl.tokens(B, seed)
+
+
+def _run(dl, B, rule_r, rule_s=None, batch_index=0, tokens=None, **kw):
+    xh, xd = _tokens(dl, B, batch_index)
+    rep = parity.compare(dl, xh, xd, rule_r, rule_s, tokens=tokens, **kw)
+    print(f"{dl.shape.name} B={B} {rule_r} {rule_s}: {rep}")
+    return rep
+
+
+# ---------------------------------------------------------------------------------------------
+def test_device_generator_matches_host():
+    for dt, tdt in ((synth.BF16, torch.bfloat16), (synth.F32, torch.float32)):
+        for seed, tid, off, std in ((0, 3, 0, 0.5), (7, 5, 123456789, 0.02), (1, 1, 17, 1.0)):
+            n = 3_000_001
+            d = torch.empty(n, dtype=tdt, device="cuda")
+            synth.fill_cuda(d, seed, tid, off, std)
+            h = synth.fill_host(n, seed, tid, off, std, dt)
+            got = d.view(torch.int16 if dt == synth.BF16 else torch.int32).cpu().numpy()
+            want = h.view(np.int16 if dt == synth.BF16 else np.int32)
+            assert np.array_equal(got, want), f"device/host generator differ ({dt}, {seed}, {tid})"
+
+
+# ---------------------------------------------------------------------------------------------
+@pytest.fixture(scope="module")
+def tiny():
+    dl = DeviceLayer(synth.TINY, max_tokens=64)
+    yield dl
+    dl.close()
+
+
+@pytest.mark.parametrize("B", [4, 1, 2, 3, 7, 16, 64])
+def test_tiny_fp32(tiny, B):
+    _run(tiny, B, ("topk", 0.5))
+
+
+@pytest.mark.parametrize("s", [0.0, 0.9, 1.0, 0.29])
+def test_tiny_sparsity(tiny, s):
+    _run(tiny, 16, ("topk", s), batch_index=3)
+
+
+def test_tiny_threshold(tiny):
+    shape = tiny.shape
+    layer = oracle.Layer(shape, synth.host_tensor(shape, "router"),
+                         parity.host_inputs(shape, range(shape.n_routed)))
+    t, _ = layer.calibrate(synth.host_tokens(shape, 256, synth.calib_seed(shape)), 0.5)
+    _run(tiny, 16, ("threshold", float(np.float32(t))), batch_index=5)
+    _run(tiny, 8, ("threshold", -np.inf), batch_index=6)
+    _run(tiny, 8, ("threshold", np.inf), batch_index=6)
+
+
+def test_tiny_identical_tokens(tiny):
+    # every token routes to the same experts: T_e = B spans several token tiles
+    xh, _ = _tokens(tiny, 1, 9)
+    xh = np.repeat(xh, 24, axis=0)
+    xd = torch.from_numpy(xh).cuda()
+    rep = parity.compare(tiny, xh, xd, ("topk", 0.5))
+    print("identical tokens:", rep)
+
+
+def test_tiny_ties():
+    """Tied router rows and tied gate rows: lower index wins on both sides, exactly."""
+    shape = synth.TINY
+    dl = DeviceLayer(shape, max_tokens=16)
+    try:
+        router = synth.host_tensor(shape, "router").copy()
+        router[5] = router[2]
+        dl.router[5] = dl.router[2]
+        experts = parity.host_inputs(shape, range(shape.n_routed))
+        for e in range(shape.n_routed):
+            g = experts[e][0].copy()
+            g[40] = g[7]
+            g[300] = g[7]
+            experts[e] = (g, experts[e][1], experts[e][2])
+            dl.gate[e, 40] = dl.gate[e, 7]
+            dl.gate[e, 300] = dl.gate[e, 7]
+        xh, _ = _tokens(dl, 8, 2)
+        # tokens aligned with router row 2 make experts 2 and 5 tie at the top
+        xh = xh.copy()
+        xh[:4] = (router[2][None, :] * 40).astype(np.float32)
+        xd = torch.from_numpy(xh).cuda()
+        rep = parity.compare(dl, xh, xd, ("topk", 0.5), expert_cache=experts, router_host=router)
+        dbg = dl.debug(8)
+        for t in range(4):
+            assert list(dbg["idx"][t][:2]) == [2, 5]
+        print("ties:", rep)
+    finally:
+        dl.close()
+
+
+def test_zero_tokens_and_errors(tiny):
+    x = torch.empty((0, tiny.shape.hidden), dtype=torch.float32, device="cuda")
+    out = tiny.forward(x, ("topk", 0.5))
+    assert out.shape[0] == 0
+    # a NaN token sets the device error word; the context stays usable
+    xh, xd = _tokens(tiny, 4, 0)
+    xd[1, 3] = float("nan")
+    tiny.forward(xd, ("topk", 0.5))
+    st, code = moe_get_error(tiny.h)
+    assert st == MOE_ERR_DEVICE and code in (1, 2)
+    st, code = moe_get_error(tiny.h)
+    assert st == MOE_OK and code == 0
+    _run(tiny, 4, ("topk", 0.5))
+
+
+# ---------------------------------------------------------------------------------------------
+@pytest.fixture(scope="module")
+def olmoe():
+    dl = DeviceLayer(synth.OLMOE, max_tokens=256)
+    yield dl
+    dl.close()
+
+
+@pytest.mark.parametrize("B", [1, 4, 16])
+@pytest.mark.parametrize("s", [0.0, 0.5, 0.9])
+def test_olmoe(olmoe, B, s):
+    _run(olmoe, B, ("topk", s), batch_index=B)
+
+
+def test_olmoe_full_batch(olmoe):
+    cache = {}
+    _run(olmoe, 256, ("topk", 0.5), batch_index=7, tokens=np.arange(0, 256, 8), expert_cache=cache)
+    _run(olmoe, 64, ("topk", 0.9), batch_index=8, expert_cache=cache)
+
+
+# ---------------------------------------------------------------------------------------------
+@pytest.fixture(scope="module")
+def dsv2l():
+    dl = DeviceLayer(synth.DSV2L, max_tokens=64)
+    yield dl
+    dl.close()
+
+
+@pytest.mark.parametrize("B", [1, 16, 64])
+@pytest.mark.parametrize("s,s_sh", [(0.0, 0.0), (0.5, 0.0), (0.9, 0.5), (0.9, 0.0)])
+def test_dsv2l(dsv2l, B, s, s_sh):
+    tokens = None if B <= 16 else np.arange(0, B, 4)
+    _run(dsv2l, B, ("topk", s), ("topk", s_sh), batch_index=B, tokens=tokens)
+
+
+# ---------------------------------------------------------------------------------------------
+@pytest.fixture(scope="module")
+def gptoss():
+    dl = DeviceLayer(synth.GPTOSS, max_tokens=64)
+    yield dl
+    dl.close()
+
+
+@pytest.mark.parametrize("B", [1, 8, 32, 64])
+@pytest.mark.parametrize("s", [0.0, 0.5, 0.9])
+def test_gptoss(gptoss, B, s):
+    tokens = None if B <= 8 else np.arange(0, B, 4)
+    _run(gptoss, B, ("topk", s), batch_index=B, tokens=tokens)
+
+
+@pytest.mark.parametrize("s", [0.5, 0.9])
+def test_gptoss_threshold(gptoss, s):
+    shape = gptoss.shape
+    gates = {e: (synth.host_tensor(shape, "gate", e), None, None) for e in range(shape.n_routed)}
+    layer = oracle.Layer(shape, synth.host_tensor(shape, "router"), gates)
+    t, n = layer.calibrate(synth.host_tokens(shape, 1024, synth.calib_seed(shape)), s)
+    print(f"calibrated t={t:.6g} over {n} scores for s={s}")
+    _run(gptoss, 32, ("threshold", float(np.float32(t))), batch_index=40 + int(s * 10),
+         tokens=np.arange(0, 32, 2))
+
+
+# ---------------------------------------------------------------------------------------------
+@pytest.fixture(scope="module")
+def llama4():
+    dl = DeviceLayer(synth.LLAMA4, max_tokens=256)
+    yield dl
+    dl.close()
+
+
+@pytest.mark.parametrize("B", [1, 2, 8])
+@pytest.mark.parametrize("s", [0.0, 0.5, 0.9])
+def test_llama4(llama4, B, s):
+    _run(llama4, B, ("topk", s), ("topk", s), batch_index=B)
+
+
+def test_llama4_large_batch(llama4):
+    shared = parity.host_shared(llama4.shape)
+    cache = {}
+    _run(llama4, 256, ("topk", 0.9), ("topk", 0.9), batch_index=99, tokens=[0, 77, 255],
+         shared_weights=shared, expert_cache=cache)
+    _run(llama4, 64, ("topk", 0.5), ("topk", 0.5), batch_index=98, tokens=[1, 33, 63],
+         shared_weights=shared, expert_cache=cache)
