@@ -1,0 +1,445 @@
+"""Benchmark of the sparse-expert MoE FFN decode layer on B200.
+
+One step = one layer call (router, gate, selection, sparse up/down, output cast) on one batch
+of synthetic decode tokens.  Default workload: the OLMoE-shaped bf16 layer (H2048, 64 experts,
+top-8, I1024) at 16 tokens and 90 % intra-expert sparsity; ``--sweep`` adds the batch x
+sparsity grid (1..256 tokens, s = 0 / 0.5 / 0.9).  L2 is flushed (a 2x-L2 buffer is written)
+before every timed step and the token batch rotates through a pool of 32.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cuda|reference]
+
+Multi-GPU: one process per GPU (torchrun); each rank runs the layer on its own token batches
+(independent decode streams, no data-path collective), so per-GPU work is fixed: weak scaling.
+``--impl reference`` times the fp64 CPU oracle on the host cores on a bounded sample of the
+same workload (rank 0 only).
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer decode tokens/sec and HBM GB/s vs roofline at batch 1–256, sparsity 0/50/90%"
+UNIT = "tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
+    ap.add_argument("--workload", default="olmoe")
+    ap.add_argument("--batch", type=int, default=16)
+    ap.add_argument("--sparsity", type=float, default=0.9)
+    ap.add_argument("--sweep", dest="sweep", action="store_true", default=None)
+    ap.add_argument("--no-sweep", dest="sweep", action="store_false")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target host time of the oracle sample")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------------------------
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9 and parts[1].isdigit():
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        return {"sm_mhz": statistics.median(int(r[1]) for r in rows),
+                "sm_max_mhz": max(int(r[2]) for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------------------------
+def algorithmic_bytes(shape, dbg, B):
+    """Bytes the method must read per stage for one call (each touched expert's gate block
+    once, each kept row of the per-expert union once), from the call's kept lists."""
+    elt, H = shape.elt, shape.hidden
+    k, S = shape.top_k, shape.n_shared
+    union = {}
+    for t in range(B):
+        for j in range(k):
+            e = int(dbg["idx"][t][j])
+            union.setdefault(("r", e), set()).update(dbg["lists"][t][j][: dbg["cnt"][t][j]].tolist())
+        for s in range(S):
+            union.setdefault(("s", s), set()).update(
+                dbg["lists"][t][k + s][: dbg["cnt"][t][k + s]].tolist())
+    gate = sum((shape.inter if kind == "r" else shape.inter_shared) * H * elt
+               for (kind, _) in union)
+    updown = sum(len(u) * 2 * H * elt for u in union.values())
+    pairs = B * (k + S)
+    imax = max(shape.inter, shape.inter_shared if S else 0)
+    return {"router": shape.n_routed * H * elt + B * H * elt, "gate": gate,
+            "select": pairs * imax * 4, "updown": updown, "finalize": B * H * (8 + elt),
+            "rows": sum(len(u) for u in union.values())}
+
+
+def run_cuda(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    from sparse_expert_ffn_logits_b200 import (STAGES, moe_forward_host, moe_profile_stages,
+                                               sparsity)
+    from sparse_expert_ffn_logits_b200.workload import DeviceLayer
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    shape = synth.SHAPES[args.workload]
+    B, s = args.batch, args.sparsity
+    sweep_on = args.sweep if args.sweep is not None else (world == 1)
+    sweep_B = [1, 4, 16, 64, 256] if sweep_on else []
+    max_tokens = max([B] + sweep_B)
+    rule = ("topk", s)
+    dl = DeviceLayer(shape, max_tokens=max_tokens, device=dev)
+    pool_n = 32
+
+    def pool(nb):
+        return [dl.tokens(nb, synth.token_seed(shape, rank * 1000 + i)) for i in range(pool_n)]
+
+    xs = pool(B)
+    out = torch.empty_like(xs[0])
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_w = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=dev)
+    flush_r = torch.ones_like(flush_w)
+
+    class _Flush:
+        """Writes a 2x-L2 buffer, then reads another one, so that the timed step starts with
+        an L2 that holds none of the layer's data and no dirty lines to write back."""
+
+        @staticmethod
+        def zero_():
+            flush_w.zero_()
+            flush_r.sum()
+
+    flush = _Flush()
+
+    def timed(batches, rule_, steps, warmup):
+        for i in range(warmup):
+            dl.forward(batches[i % len(batches)], rule_, rule_, out=out_b[id(batches)])
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        for i in range(steps):
+            flush.zero_()
+            evs[i][0].record()
+            dl.forward(batches[i % len(batches)], rule_, rule_, out=out_b[id(batches)])
+            evs[i][1].record()
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in evs]
+
+    out_b = {id(xs): out}
+    # ---- the timed run (warm-up, barrier, K steps, barrier)
+    for i in range(args.warmup):
+        dl.forward(xs[i % pool_n], rule, rule, out=out)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    props = torch.cuda.get_device_properties(dev)
+    uuid = str(getattr(props, "uuid", "") or "")
+    clocks = ClockSampler(f"GPU-{uuid}" if uuid and not uuid.startswith("GPU-") else
+                          (uuid or str(local_rank)))
+    clocks.start()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        evs[i][0].record()
+        dl.forward(xs[i % pool_n], rule, rule, out=out)
+        evs[i][1].record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    value = world * B * args.steps / (total_ms / 1e3)
+
+    # ---- per-stage durations (kernels launched back to back, events between them)
+    stage_evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)]
+    for e in stage_evs:
+        e.record()
+    torch.cuda.synchronize()
+    moe_profile_stages(dl.h, stage_evs)
+    stage_ms = {n: [] for n in STAGES}
+    nprof = min(args.steps, 20)
+    for i in range(nprof):
+        flush.zero_()
+        dl.forward(xs[i % pool_n], rule, rule, out=out)
+        torch.cuda.synchronize()
+        for j, n in enumerate(STAGES):
+            stage_ms[n].append(stage_evs[j].elapsed_time(stage_evs[j + 1]))
+    moe_profile_stages(dl.h, None)
+    abytes = {n: 0.0 for n in STAGES}
+    nb = min(pool_n, nprof)
+    for i in range(nb):
+        dl.forward(xs[i], rule, rule, out=out)
+        ab = algorithmic_bytes(shape, dl.debug(B), B)
+        for n in STAGES:
+            abytes[n] += ab[n] / nb
+    stage_avg = {n: statistics.mean(v) for n, v in stage_ms.items()}
+    dom = max(STAGES, key=lambda n: stage_avg[n])
+    peak, peak_kind = peaks()
+    achieved = abytes[dom] / (stage_avg[dom] / 1e3) / 1e9
+    layer_bytes = sum(abytes[n] for n in ("router", "gate", "updown"))
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            tr = json.load(f).get(f"{args.workload}:B{B}:s{s}:{dom}")
+        traffic = tr
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
+                "peak_source": f"hbm copy, {peak_kind}", "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic,
+                "algorithmic_bytes_per_launch": int(abytes[dom]),
+                "launch_us": round(stage_avg[dom] * 1e3, 2),
+                "stages_us": {n: round(v * 1e3, 2) for n, v in stage_avg.items()},
+                "layer": {"algorithmic_bytes": int(layer_bytes),
+                          "gbs": round(layer_bytes / (total_ms / args.steps / 1e3) / 1e9, 1),
+                          "frac": round(layer_bytes / (total_ms / args.steps / 1e3) / 1e9 / peak, 4)}}
+
+    # ---- end to end through the host-buffer C call (pinned host memory, copies inside)
+    xh = [x.cpu().pin_memory() for x in xs[:8]]
+    oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    sr = sparsity(rule)
+    ss = sparsity(rule) if shape.n_shared else None
+    for i in range(args.warmup):
+        moe_forward_host(dl.h, xh[i % 8], B, dl.router, dl.routed, dl.shared, sr, ss, oh)
+    torch.cuda.synchronize()
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        e2e_ev[i][0].record()
+        moe_forward_host(dl.h, xh[i % 8], B, dl.router, dl.routed, dl.shared, sr, ss, oh)
+        e2e_ev[i][1].record()
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    io_bytes = B * shape.hidden * shape.elt
+    e2e = {"value": round(world * B * args.steps / (e2e_ms / 1e3), 1), "unit": UNIT,
+           "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes,
+           "api": "moe_forward_host"}
+
+    # ---- sweep (rank 0, single GPU)
+    sweep = []
+    if sweep_on and rank == 0:
+        for sb in sweep_B:
+            bx = pool(sb)
+            out_b[id(bx)] = torch.empty_like(bx[0])
+            row = {}
+            for ss_ in (0.0, 0.5, 0.9):
+                r_ = ("topk", ss_)
+                ms = timed(bx, r_, 20, 3)
+                med = statistics.median(ms)
+                nbytes = 0.0
+                for i in range(4):
+                    dl.forward(bx[i], r_, r_, out=out_b[id(bx)])
+                    ab = algorithmic_bytes(shape, dl.debug(sb), sb)
+                    nbytes += (ab["router"] + ab["gate"] + ab["updown"]) / 4
+                gbs = nbytes / (med / 1e3) / 1e9
+                row[ss_] = med
+                sweep.append({"batch": sb, "sparsity": ss_, "us": round(med * 1e3, 1),
+                              "tokens_per_s": round(sb / (med / 1e3), 1),
+                              "active_bytes": int(nbytes), "gbs": round(gbs, 1),
+                              "frac": round(gbs / peak, 4)})
+            sweep[-1]["speedup_s0.9_vs_s0"] = round(row[0.0] / row[0.9], 3)
+            del out_b[id(bx)]
+
+    # ---- CPU baseline: the oracle, as it stands, on a bounded sample (rank 0, N = 1)
+    cpu = None
+    if rank == 0 and world == 1:
+        cpu = cpu_baseline(shape, B, rule, args.cpu_seconds)
+
+    dl.close()
+    line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total_ms / args.steps, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": shape.dtype, "data": "synthetic",
+            "config": {"workload": f"{shape.name}-shaped MoE layer", "hidden": shape.hidden,
+                       "experts": shape.n_routed, "top_k": shape.top_k, "inter": shape.inter,
+                       "shared": shape.n_shared, "batch_per_gpu": B, "global_batch": B * world,
+                       "sparsity": s, "selection": "top-K per (token, expert)",
+                       "l2": "flushed before every step: a 2x-L2 buffer written, then another "
+                             "2x-L2 buffer read (clean lines, none of the layer's)",
+                       "token_pool": pool_n, "parallelism": f"replicas x{world}"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": 5 * args.steps, "clocks": clock_info}
+    if sweep:
+        line["sweep"] = sweep
+    return line
+
+
+# ---------------------------------------------------------------------------------------------
+def cpu_baseline(shape, B, rule, seconds):
+    """Times the fp64 oracle (all host cores) on whole token batches of the benchmark's stream,
+    batch after batch, until about `seconds` of oracle time has been spent."""
+    import oracle
+    import synth
+    router = synth.host_tensor(shape, "router")
+    rl = oracle.Layer(shape, router, {}, [])
+    shared = [(synth.host_tensor(shape, "sh_gate", j), synth.host_tensor(shape, "sh_up", j),
+               synth.host_tensor(shape, "sh_down", j)) for j in range(shape.n_shared)]
+    cache = {}
+    done_tok, spent, nb = 0, 0.0, 0
+    while spent < seconds and nb < 64:
+        x = synth.host_tokens(shape, B, synth.token_seed(shape, nb))
+        _, idx, _ = rl.route(x)
+        need = sorted(set(int(e) for e in idx.ravel()))
+        for e in need:
+            if e not in cache:
+                cache[e] = (synth.host_tensor(shape, "gate", e), synth.host_tensor(shape, "up", e),
+                            synth.host_tensor(shape, "down", e))
+        lay = oracle.Layer(shape, router, {e: cache[e] for e in need}, shared)
+        t0 = time.perf_counter()
+        lay.forward(x, rule, rule)
+        spent += time.perf_counter() - t0
+        done_tok += B
+        nb += 1
+    return {"value": round(done_tok / spent, 3), "unit": UNIT, "cores": oracle.threads(),
+            "kind": "oracle",
+            "sample": f"{nb} batches of {B} tokens (token streams 1..{nb}), whole layer in fp64, "
+                      f"{spent:.1f} s of oracle time"}
+
+
+def run_reference(args):
+    """The benchmark's reference arm: the fp64 CPU oracle, timed on the host cores."""
+    import synth
+    shape = synth.SHAPES[args.workload]
+    B, rule = args.batch, ("topk", args.sparsity)
+    per_step = max(1.0, args.cpu_seconds / max(1, args.steps + args.warmup) * 4)
+    import oracle
+    x_all = [synth.host_tokens(shape, B, synth.token_seed(shape, i)) for i in range(4)]
+    router = synth.host_tensor(shape, "router")
+    rl = oracle.Layer(shape, router, {}, [])
+    shared = [(synth.host_tensor(shape, "sh_gate", j), synth.host_tensor(shape, "sh_up", j),
+               synth.host_tensor(shape, "sh_down", j)) for j in range(shape.n_shared)]
+    cache = {}
+
+    def layer_for(x):
+        _, idx, _ = rl.route(x)
+        need = sorted(set(int(e) for e in idx.ravel()))
+        for e in need:
+            if e not in cache:
+                cache[e] = (synth.host_tensor(shape, "gate", e), synth.host_tensor(shape, "up", e),
+                            synth.host_tensor(shape, "down", e))
+        return oracle.Layer(shape, router, {e: cache[e] for e in need}, shared)
+
+    # tokens per step: sized so the whole run stays within a few minutes
+    probe = layer_for(x_all[0][:1])
+    t0 = time.perf_counter()
+    probe.forward(x_all[0][:1], rule, rule)
+    one = time.perf_counter() - t0
+    ntok = int(max(1, min(B, per_step / max(one, 1e-6))))
+    layers = [layer_for(x[:ntok]) for x in x_all]
+    for i in range(args.warmup):
+        layers[i % 4].forward(x_all[i % 4][:ntok], rule, rule)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        layers[i % 4].forward(x_all[i % 4][:ntok], rule, rule)
+    dt = time.perf_counter() - t0
+    value = ntok * args.steps / dt
+    sample = f"{ntok} of {B} tokens per step, whole layer in fp64"
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{shape.name}-shaped MoE layer", "hidden": shape.hidden,
+                       "experts": shape.n_routed, "top_k": shape.top_k, "inter": shape.inter,
+                       "shared": shape.n_shared, "batch_per_gpu": B, "sparsity": args.sparsity,
+                       "parallelism": "host cores"},
+            "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": oracle.threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_cuda(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -148,6 +148,21 @@ moe_status moe_forward_host(moe_handle* h, const void* x_host, int n_tokens, con
 moe_status moe_debug_lists(moe_handle* h, int n_tokens, int* idx, float* w, float* logits,
                            int* cnt, int* lists, float* act, void* stream);
 
+/* Stage timing.  events = MOE_STAGE_EVENTS cudaEvent_t handles (as void*), or NULL to turn
+ * timing off.  While set, every moe_forward records events[0] before its first kernel and
+ * events[i] after its i-th kernel (1 router+top-k+grouping, 2 gate, 3 select, 4 up/down,
+ * 5 output cast), and launches the kernels without programmatic overlap so that the interval
+ * between consecutive events is that kernel alone.  The handle keeps the event handles, not
+ * copies; the caller owns and destroys them. */
+#define MOE_STAGE_EVENTS 6
+moe_status moe_profile_stages(moe_handle* h, void* const* events, int n_events);
+
+/* Phase timestamps of the last calls made while stage timing was on (%globaltimer ns, 0 where a
+ * point was not reached): host[(kernel * 1024 + cta) * 8 + point] for kernel 0..4 in launch
+ * order and the first 1024 CTAs.  Synchronises the device, copies min(n, 5*1024*8) values into
+ * host memory, then clears the device buffer. */
+moe_status moe_read_trace(moe_handle* h, unsigned long long* host, size_t n);
+
 /* Synchronises the device, reads and clears the device error word.  Returns MOE_ERR_DEVICE
  * (code in *device_code: 1 = NaN router logit, 2 = NaN activation) if it was set, else MOE_OK
  * with *device_code = 0. */

@@ -50,8 +50,10 @@ _LIB = None
 
 # C entry points declared in include/moe.h
 EXPORTS = ("moe_create", "moe_packed_bytes", "moe_pack_experts", "moe_forward",
-           "moe_forward_host", "moe_debug_lists", "moe_get_error", "moe_destroy",
-           "moe_status_string")
+           "moe_forward_host", "moe_debug_lists", "moe_profile_stages", "moe_read_trace",
+           "moe_get_error", "moe_destroy", "moe_status_string")
+MOE_STAGE_EVENTS = 6
+STAGES = ("router", "gate", "select", "updown", "finalize")
 
 
 def _lib():
@@ -72,6 +74,8 @@ def _lib():
         lib.moe_forward.argtypes = fwd
         lib.moe_forward_host.argtypes = fwd
         lib.moe_debug_lists.argtypes = [P, I, P, P, P, P, P, P, P]
+        lib.moe_profile_stages.argtypes = [P, ctypes.POINTER(P), I]
+        lib.moe_read_trace.argtypes = [P, P, ctypes.c_size_t]
         lib.moe_get_error.argtypes = [P, ctypes.POINTER(I)]
         lib.moe_destroy.argtypes = [P]
         lib.moe_status_string.argtypes = [I]
@@ -170,6 +174,25 @@ def moe_debug_lists(h, n_tokens, idx=None, w=None, logits=None, cnt=None, lists=
     _check(_lib().moe_debug_lists(ctypes.c_void_p(h), int(n_tokens), _ptr(idx), _ptr(w),
                                   _ptr(logits), _ptr(cnt), _ptr(lists), _ptr(act),
                                   _stream(stream)), "moe_debug_lists")
+
+
+def moe_profile_stages(h, events):
+    """events: MOE_STAGE_EVENTS torch.cuda.Event objects (timing on) or None (timing off)."""
+    if events is None:
+        _check(_lib().moe_profile_stages(ctypes.c_void_p(h), None, 0), "moe_profile_stages")
+        return
+    arr = (ctypes.c_void_p * len(events))(*[ev.cuda_event for ev in events])
+    _check(_lib().moe_profile_stages(ctypes.c_void_p(h), arr, len(events)),
+           "moe_profile_stages")
+
+
+def moe_read_trace(h):
+    """Phase timestamps as a numpy array [5 kernels][1024 CTAs][8 points] (ns, 0 = not reached)."""
+    import numpy as np
+    buf = np.zeros(5 * 1024 * 8, dtype=np.uint64)
+    _check(_lib().moe_read_trace(ctypes.c_void_p(h), ctypes.c_void_p(buf.ctypes.data), buf.size),
+           "moe_read_trace")
+    return buf.reshape(5, 1024, 8)
 
 
 def moe_get_error(h):

@@ -15,6 +15,7 @@ constexpr int kMaxTopK = 16;
 constexpr int kMaxShared = 8;
 constexpr int kMaxRouted = 512;
 constexpr int kMaxTokens = 1024;
+constexpr int kMaxHsplit = 16;     // router slices of H
 
 // device error word codes
 constexpr int kErrNanLogit = 1;
@@ -31,11 +32,33 @@ struct Slot {
   int pad0, pad1;
 };
 
+// A slot written by an earlier kernel of the same call, read through L2 (never a stale L1 line).
+__device__ __forceinline__ Slot load_slot(const Slot* s) {
+  const int4 a = __ldcg(reinterpret_cast<const int4*>(s));
+  const int4 b = __ldcg(reinterpret_cast<const int4*>(s) + 1);
+  Slot r;
+  r.kind = a.x; r.expert = a.y; r.T = a.z; r.q0 = a.w;
+  r.I = b.x; r.item0 = b.y; r.pad0 = b.z; r.pad1 = b.w;
+  return r;
+}
+
+// Index j of the last table entry with tab[j].w <= item (entries ascending in .w).
+__device__ __forceinline__ int find_item_slot(const int4* tab, int n, int item) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tab[mid].w <= item) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
 // meta words written by the router kernel
 enum { kMetaSlots = 0, kMetaPairs = 1, kMetaGateItems = 2, kMetaTouched = 3, kMetaWords = 8 };
 
 struct FwdParams {
   int H, E, k, S, I, Ish, B, Imax;
+  int Bmax;         // max_tokens of the handle
+  int hsplit;       // router slices of H
   int route;
   int sel_mode[2];  // [0] routed, [1] shared: 0 top-K, 1 threshold
   int sel_K[2];
@@ -49,6 +72,7 @@ struct FwdParams {
   void* out;
   // workspace
   float* logits;       // [Bmax][E]
+  float* logit_part;   // [kMaxHsplit][Bmax][E] partial router logits
   int* topk_idx;       // [Bmax][k]
   float* topk_w;       // [Bmax][k]
   int* pair_index;     // [Bmax][k+S]
@@ -69,7 +93,28 @@ struct FwdParams {
   int* ucnt;           // [E+S]
   float* out_acc;      // [Bmax][H]
   int* err;            // device error word
+  const void* zero_row;  // H zero elements (source of the copies of absent tokens)
+  unsigned long long* trace;  // per-CTA phase timestamps (nullptr: tracing off)
 };
+
+// Phase timestamps for tracing: kernel k, CTA b, point i (i < kTracePoints).
+constexpr int kTraceKernels = 5, kTraceCtas = 1024, kTracePoints = 8;
+__device__ __forceinline__ void trace_point(const unsigned long long* tr_base, int kernel, int i) {
+  if (tr_base && threadIdx.x == 0 && blockIdx.x + blockIdx.y * gridDim.x < kTraceCtas) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    const_cast<unsigned long long*>(tr_base)[((size_t)kernel * kTraceCtas + blockIdx.x +
+                                              blockIdx.y * gridDim.x) * kTracePoints + i] = t;
+  }
+}
+
+// Slot table in shared memory as int4 {expert | kind << 16, T, q0, item0}.
+__device__ __forceinline__ void load_slot_table(const FwdParams& p, int n_slots, int4* s_tab) {
+  for (int j = threadIdx.x; j < n_slots; j += blockDim.x) {
+    const Slot s = load_slot(&p.slots[j]);
+    s_tab[j] = make_int4(s.expert | (s.kind << 16), s.T, s.q0, s.item0);
+  }
+}
 
 // ---------------------------------------------------------------------------------------------
 // Programmatic dependent launch: a kernel launched with the programmatic-serialization attribute

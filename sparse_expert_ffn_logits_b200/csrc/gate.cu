@@ -3,58 +3,270 @@
 // The gate is the part of an expert that cannot be skipped: it is what scores the neurons
 // ("Uncovering Intra-expert Activation Sparsity ...", technical summary, Methodology: the gate
 // projection runs densely to determine the activation scores).  Every evaluated expert's gate
-// block [I][H] is read from HBM once per token tile.
+// block [I][H] is read from HBM once per tile of 8 of its tokens.
 //
-// Persistent grid over work items (slot, row group of 16 neurons, token tile of 8 pairs),
-// row group outer so that the token tiles of one row group run at the same time and share the
-// rows through L2.  In an item the 8 warps split H; their partial 16x8 fragments are summed in
-// shared memory and warp 0 writes act[q][n] = SiLU(g) in fp32.
+// Work item = (slot, token tile of 8 pairs, group of 16 neurons), ordered slot, token tile,
+// neuron group; each CTA takes a contiguous range of items.  Output act[q][n] = SiLU(g) in fp32.
+//
+// bf16: one persistent CTA per SM with three roles.
+//   meta warp    walks the items ahead of the others (at most kMetaRing): resolves each item's
+//                rows and pairs into a small shared-memory ring and, when the token tile
+//                changes, bulk-copies the 8 token rows into one of two token-tile buffers;
+//   copier warp  streams the item's 16 gate rows, kc columns at a time, into a ring of
+//                shared-memory stages (bulk asynchronous copies completed on mbarriers);
+//   8 consumer warps  split each stage's columns, multiply on the tensor cores against the
+//                token tile, and sum their partial 16x8 tiles at the end of the item.
+// Consumers issue no global load: every latency is taken by a warp that runs ahead.
+// fp32: a plain CUDA-core variant (register loads, same fragment layout).
 #include "kernels.h"
 #include "tile.cuh"
+#include "tma.cuh"
 
 namespace moe {
 namespace {
 
 constexpr int kMaxSlots = kMaxRouted + kMaxShared;
+constexpr int kRingThreads = kThreads + 64;  // 8 consumer warps, copier, meta
+constexpr int kCopier = kWarps, kMetaWarp = kWarps + 1;
 
-template <typename T>
-__global__ void __launch_bounds__(kThreads) gate_kernel(FwdParams p) {
+struct GateMeta {
+  const __nv_bfloat16* rows;  // first of the item's 16 consecutive gate rows
+  int q0;                     // pair index of the tile's first token
+  int nt;                     // valid tokens in the tile (1..8)
+  int n0;                     // first neuron
+  int xb, xpar, xlast;        // token tile buffer, its fill phase, last item using it
+};
+
+__global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, Ring rc) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ int4 s_tab[kMaxSlots];
+  __shared__ GateMeta s_meta[kMetaRing];
+  __shared__ int s_abort;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty = full + rc.ns;
+  uint64_t* mfull = empty + rc.ns;
+  uint64_t* mempty = mfull + kMetaRing;
+  uint64_t* xfull = mempty + kMetaRing;
+  uint64_t* xempty = xfull + 2;
+  float(*red)[kWarps][4][32] = reinterpret_cast<float(*)[kWarps][4][32]>(smem + kBarBytes);
+  unsigned char* xbuf = smem + kBarBytes + kRedBytes;
+  unsigned char* ring = xbuf + rc.nxb * rc.xs_bytes;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
+  trace_point(p.trace, 1, 0);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < rc.ns; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kWarps);
+    }
+    for (int i = 0; i < kMetaRing; ++i) {
+      mbar_init(&mfull[i], 1);
+      mbar_init(&mempty[i], kWarps + 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&xfull[i], 1);
+      mbar_init(&xempty[i], kWarps);
+    }
+    s_abort = 0;
+    for (int i = 0; i < kMetaRing; ++i) {
+      s_meta[i].rows = static_cast<const __nv_bfloat16*>(p.gate_r);
+      s_meta[i].q0 = s_meta[i].nt = s_meta[i].n0 = 0;
+      s_meta[i].xb = s_meta[i].xpar = s_meta[i].xlast = 0;
+    }
+    mbar_init_fence();
+  }
+  pdl_trigger();
+  pdl_wait();
+  trace_point(p.trace, 1, 1);
+  const int n_slots = ld_cg(&p.meta[kMetaSlots]);
+  const int n_items = ld_cg(&p.meta[kMetaGateItems]);
+  load_slot_table(p, n_slots, s_tab);
+  __syncthreads();
+  const int i0 = (int)((long long)blockIdx.x * n_items / gridDim.x);
+  const int i1 = (int)((long long)(blockIdx.x + 1) * n_items / gridDim.x);
+  const int H = p.H;
+  volatile int* abort = &s_abort;
+
+  if (warp == kMetaWarp) {
+    // ---------------- meta: item records and token tiles, ahead of everyone
+    if (i0 >= i1) return;
+    int j = find_item_slot(s_tab, n_slots, i0);
+    int I = (s_tab[j].x >> 16) ? p.Ish : p.I;
+    int local = i0 - s_tab[j].w;
+    int tt = local / (I / kTileRows), rg = local % (I / kTileRows);
+    int key = -1, xb = rc.nxb - 1;
+    int xuse[2] = {0, 0};
+    for (int item = i0, mi = 0; item < i1; ++item, ++mi) {
+      const int m = mi % kMetaRing;
+      if (!mbar_wait(&mempty[m], ((mi / kMetaRing) & 1) ^ 1, abort, p.err)) break;
+      const int4 sl = s_tab[j];
+      const int kind = sl.x >> 16, ex = sl.x & 0xffff, T = sl.y, q0 = sl.z;
+      const int nt = min(kTileTok, T - tt * kTileTok);
+      int xpar;
+      if (j * 1024 + tt != key) {
+        key = j * 1024 + tt;
+        xb = (xb + 1) % rc.nxb;
+        if (!mbar_wait(&xempty[xb], (xuse[xb] & 1) ^ 1, abort, p.err)) break;
+        xpar = xuse[xb] & 1;
+        xuse[xb]++;
+        if (lane == 0) mbar_arrive_expect_tx(&xfull[xb], kTileTok * H * 2);
+        __syncwarp();
+        if (lane < kTileTok) {
+          const void* src = p.zero_row;
+          if (lane < nt)
+            src = static_cast<const __nv_bfloat16*>(p.x) +
+                  (size_t)__ldcg(&p.pair_token[q0 + tt * kTileTok + lane]) * H;
+          bulk_g2s(xbuf + xb * rc.xs_bytes + lane * rc.xs_stride, src, H * 2, &xfull[xb]);
+        }
+      } else {
+        xpar = (xuse[xb] - 1) & 1;
+      }
+      // the next item, to know whether this one is the last on its token tile
+      int nj = j, ntt = tt, nrg = rg + 1;
+      if (nrg == I / kTileRows) {
+        nrg = 0;
+        ++ntt;
+        if (ntt * kTileTok >= T) {
+          ntt = 0;
+          ++nj;
+        }
+      }
+      const bool last = item + 1 == i1 || nj * 1024 + ntt != key;
+      if (lane == 0) {
+        const __nv_bfloat16* base =
+            kind == 0 ? static_cast<const __nv_bfloat16*>(p.gate_r) + (size_t)ex * p.I * H
+                      : static_cast<const __nv_bfloat16*>(p.gate_s) + (size_t)ex * p.Ish * H;
+        GateMeta gm;
+        gm.rows = base + (size_t)rg * kTileRows * H;
+        gm.q0 = q0 + tt * kTileTok;
+        gm.nt = nt;
+        gm.n0 = rg * kTileRows;
+        gm.xb = xb;
+        gm.xpar = xpar;
+        gm.xlast = last;
+        s_meta[m] = gm;
+        mbar_arrive(&mfull[m]);
+      }
+      __syncwarp();
+      if (nj != j && nj < n_slots) I = (s_tab[nj].x >> 16) ? p.Ish : p.I;
+      j = nj;
+      tt = ntt;
+      rg = nrg;
+    }
+    // no token-tile copy may still be landing in shared memory when the CTA exits
+    for (int b = 0; b < rc.nxb; ++b)
+      if (xuse[b] > 0) mbar_drain(&xfull[b], (xuse[b] - 1) & 1);
+    return;
+  }
+
+  if (warp == kCopier) {
+    // ---------------- copier: the item's 16 rows, kc columns per stage, one bulk copy per row
+    const uint32_t piece = rc.kc * 2;
+    int it = 0;
+    for (int item = i0, mi = 0; item < i1 && !*abort; ++item, ++mi) {
+      const int m = mi % kMetaRing;
+      if (!mbar_wait(&mfull[m], (mi / kMetaRing) & 1, abort, p.err)) break;
+      const __nv_bfloat16* row = s_meta[m].rows + (size_t)(lane & 15) * H;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&mempty[m]);
+      for (int kc = 0; kc < rc.nk; ++kc, ++it) {
+        const int st = it % rc.ns;
+        if (!mbar_wait(&empty[st], ((it / rc.ns) & 1) ^ 1, abort, p.err)) break;
+        if (lane == 0) mbar_arrive_expect_tx(&full[st], kTileRows * piece);
+        __syncwarp();
+        if (lane < kTileRows)
+          bulk_g2s(ring + (size_t)st * rc.stage_bytes + lane * rc.rs_a, row + kc * rc.kc, piece,
+                   &full[st]);
+      }
+    }
+    for (int k = it - 1; k >= 0 && k >= it - rc.ns; --k) mbar_drain(&full[k % rc.ns], (k / rc.ns) & 1);
+    return;
+  }
+
+  // ---------------- consumers
+  int it = 0, ib = 0;
+  bool nan_seen = false;
+  const int nblk = rc.kc / 32;
+  for (int item = i0, mi = 0; item < i1; ++item, ++mi) {
+    const int m = mi % kMetaRing;
+    mbar_wait(&mfull[m], (mi / kMetaRing) & 1, abort, p.err);
+    const GateMeta gm = s_meta[m];
+    const int xb = min(max(gm.xb, 0), rc.nxb - 1);  // a record is trusted only without abort
+    mbar_wait(&xfull[xb], gm.xpar, abort, p.err);
+    const unsigned char* xrow = xbuf + xb * rc.xs_bytes + g * rc.xs_stride;
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int kc = 0; kc < rc.nk; ++kc, ++it) {
+      const int st = it % rc.ns;
+      mbar_wait(&full[st], (it / rc.ns) & 1, abort, p.err);
+      const unsigned char* stage = ring + (size_t)st * rc.stage_bytes;
+      for (int b = warp; b < nblk; b += kWarps) {
+        const int col = (b * 32 + t * 8) * 2;
+        const uint4 a0 = lds128(stage + g * rc.rs_a + col);
+        const uint4 a1 = lds128(stage + (g + 8) * rc.rs_a + col);
+        const uint4 xv = lds128(xrow + kc * rc.kc * 2 + col);
+        mma_16816(d, a0.x, a1.x, a0.y, a1.y, xv.x, xv.y);
+        mma_16816(d, a0.z, a1.z, a0.w, a1.w, xv.z, xv.w);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+    }
+    if (lane == 0) {
+      mbar_arrive(&mempty[m]);
+      if (gm.xlast) mbar_arrive(&xempty[xb]);
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) red[ib][warp][c][lane] = d[c];
+    const int aborted = consumer_sync_or(kThreads, *abort);
+    if (threadIdx.x < 128 && !aborted) {
+      // one output per thread: fragment element (c, lane), summed over the warps in order
+      const int ln = threadIdx.x & 31, c = threadIdx.x >> 5;
+      float v = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) v += red[ib][w][c][ln];
+      const int ti = 2 * (ln & 3) + (c & 1);
+      if (ti < gm.nt) {
+        const float a = silu(v);
+        nan_seen |= isnan(a);
+        p.act[(size_t)(gm.q0 + ti) * p.Imax + gm.n0 + (ln >> 2) + (c >> 1) * 8] = a;
+      }
+    }
+    ib ^= 1;
+  }
+  if (nan_seen) set_error(p.err, kErrNanAct);
+  trace_point(p.trace, 1, 7);
+}
+
+// fp32 variant: register loads, 8 warps split H, same items.
+__global__ void __launch_bounds__(kThreads) gate_f32_kernel(FwdParams p) {
   __shared__ float red[kWarps][32][4];
-  __shared__ Slot s_slot[kMaxSlots];
-  __shared__ int s_item0[kMaxSlots];
-  __shared__ const T* s_x[kTileTok];
+  __shared__ int4 s_tab[kMaxSlots];
+  __shared__ const float* s_x[kTileTok];
   pdl_trigger();
   pdl_wait();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
   const int H = p.H, Imax = p.Imax;
   const int n_slots = ld_cg(&p.meta[kMetaSlots]);
   const int n_items = ld_cg(&p.meta[kMetaGateItems]);
-  for (int j = threadIdx.x; j < n_slots; j += blockDim.x) {
-    s_slot[j] = p.slots[j];
-    s_item0[j] = p.slots[j].item0;
-  }
+  load_slot_table(p, n_slots, s_tab);
   __syncthreads();
-  const T* x = static_cast<const T*>(p.x);
+  const float* x = static_cast<const float*>(p.x);
   bool nan_seen = false;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-    const int j = find_slot(s_item0, n_slots, item);
-    const Slot s = s_slot[j];
-    const int local = item - s.item0;
-    const int ntt = (s.T + kTileTok - 1) / kTileTok;
-    const int rg = local / ntt, tt = local % ntt;
-    const int n0 = rg * kTileRows;
+    const int j = find_item_slot(s_tab, n_slots, item);
+    const int4 sl = s_tab[j];
+    const int kind = sl.x >> 16, ex = sl.x & 0xffff, T = sl.y, q0 = sl.z;
+    const int I = kind ? p.Ish : p.I;
+    const int local = item - sl.w, tt = local / (I / kTileRows), rg = local % (I / kTileRows);
     if (threadIdx.x < kTileTok) {
       const int ti = tt * kTileTok + threadIdx.x;
-      s_x[threadIdx.x] = ti < s.T ? x + (size_t)p.pair_token[s.q0 + ti] * H : nullptr;
+      s_x[threadIdx.x] = ti < T ? x + (size_t)__ldcg(&p.pair_token[q0 + ti]) * H : nullptr;
     }
     __syncthreads();
-    const T* base = s.kind == 0
-                        ? static_cast<const T*>(p.gate_r) + (size_t)s.expert * p.I * H
-                        : static_cast<const T*>(p.gate_s) + (size_t)s.expert * p.Ish * H;
-    const T* rowA = base + (size_t)(n0 + g) * H;
-    const T* rowB = base + (size_t)(n0 + g + 8) * H;
+    const float* base = kind == 0 ? static_cast<const float*>(p.gate_r) + (size_t)ex * p.I * H
+                                  : static_cast<const float*>(p.gate_s) + (size_t)ex * p.Ish * H;
+    const int n0 = rg * kTileRows;
     float d[4] = {0.f, 0.f, 0.f, 0.f};
-    tile_dot<4>(rowA, rowB, s_x, warp, kWarps, H / 32, d);
+    tile_dot<1>(base + (size_t)(n0 + g) * H, base + (size_t)(n0 + g + 8) * H, s_x, warp, kWarps,
+                H / 32, d);
 #pragma unroll
     for (int c = 0; c < 4; ++c) red[warp][lane][c] = d[c];
     __syncthreads();
@@ -63,11 +275,10 @@ __global__ void __launch_bounds__(kThreads) gate_kernel(FwdParams p) {
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int ti = tt * kTileTok + 2 * t + (c & 1);
-        if (ti < s.T) {
-          const int n = n0 + g + (c >> 1) * 8;
+        if (ti < T) {
           const float a = silu(d[c]);
           nan_seen |= isnan(a);
-          p.act[(size_t)(s.q0 + ti) * Imax + n] = a;
+          p.act[(size_t)(q0 + ti) * Imax + n0 + g + (c >> 1) * 8] = a;
         }
       }
     }
@@ -78,20 +289,61 @@ __global__ void __launch_bounds__(kThreads) gate_kernel(FwdParams p) {
 
 }  // namespace
 
-cudaError_t launch_gate(const FwdParams& p, int dtype, const LaunchShape& ls, cudaStream_t st) {
-  if (dtype == 0)
-    return launch_pdl(gate_kernel<__nv_bfloat16>, dim3(ls.grid_gate), dim3(kThreads), 0, st, true,
-                      p);
-  return launch_pdl(gate_kernel<float>, dim3(ls.grid_gate), dim3(kThreads), 0, st, true, p);
+// Copy-ring shape for hidden size H: the widest row pieces (kc a multiple of 64 dividing H) that
+// still leave two stages, two token tiles when they fit.  Bulk copies of a few kilobytes reach
+// the HBM copy rate, copies of 1 KB reach about half of it.
+Ring make_ring(int H, int smem_budget, int static_smem) {
+  const int avail = smem_budget - static_smem - kBarBytes - kRedBytes;
+  Ring best{};
+  best.ns = 0;
+  for (int nk = 1; nk <= H / 64; ++nk) {
+    if (H % nk || (H / nk) % 64) continue;
+    Ring r;
+    r.nk = nk;
+    r.kc = H / nk;
+    r.rs_a = r.kc * 2 + 64;
+    r.rs_d = r.kc * 2 + 16;
+    r.stage_bytes = kTileRows * r.rs_a;
+    r.xs_stride = H * 2 + 64;
+    r.xs_bytes = kTileTok * r.xs_stride;
+    for (int nxb = 2; nxb >= 1; --nxb) {
+      int ns = (avail - nxb * r.xs_bytes) / r.stage_bytes;
+      if (ns > 16) ns = 16;
+      if (ns >= 2) {
+        r.nxb = nxb;
+        r.ns = ns;
+        r.smem_bytes = kBarBytes + kRedBytes + nxb * r.xs_bytes + ns * r.stage_bytes;
+        return r;
+      }
+    }
+  }
+  return best;  // ns == 0: no ring fits
 }
 
-int gate_occupancy(int dtype) {
-  int n = 0;
+cudaError_t launch_gate(const FwdParams& p, int dtype, const LaunchShape& ls, cudaStream_t st,
+                        bool pdl) {
   if (dtype == 0)
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gate_kernel<__nv_bfloat16>, kThreads, 0);
-  else
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gate_kernel<float>, kThreads, 0);
-  return n;
+    return launch_pdl(gate_tma_kernel, dim3(ls.nsm), dim3(kRingThreads), ls.ring_gate.smem_bytes,
+                      st, pdl, p, ls.ring_gate);
+  return launch_pdl(gate_f32_kernel, dim3(ls.grid_gate), dim3(kThreads), 0, st, pdl, p);
+}
+
+cudaError_t configure_gate(int dtype, int H, int smem_budget, LaunchShape* ls) {
+  if (dtype == 0) {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, gate_tma_kernel);
+    if (e != cudaSuccess) return e;
+    ls->ring_gate = make_ring(H, smem_budget, (int)fa.sharedSizeBytes + 1024);
+    if (ls->ring_gate.ns < 2) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(gate_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ls->ring_gate.smem_bytes);
+    ls->grid_gate = ls->nsm;
+    return e;
+  }
+  int n = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gate_f32_kernel, kThreads, 0);
+  ls->grid_gate = ls->nsm * (n > 0 ? n : 1);
+  return e;
 }
 
 }  // namespace moe

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include "common.cuh"
+#include "tma.cuh"
 
 namespace moe {
 
@@ -12,17 +13,24 @@ struct LaunchShape {
   int grid_gate;      // persistent grid of the gate kernel
   int grid_updown;    // persistent grid of the up/down kernel
   int grid_select;    // cap of the selection grid
+  Ring ring_gate;     // copy ring of the bf16 gate kernel
+  Ring ring_ud;       // copy ring of the bf16 up/down kernel
 };
 
 // dtype: 0 bf16, 1 fp32.  Each launcher returns the launch's cudaError_t.
 cudaError_t launch_router(const FwdParams& p, int dtype, cudaStream_t st);
-cudaError_t launch_gate(const FwdParams& p, int dtype, const LaunchShape& ls, cudaStream_t st);
-cudaError_t launch_select(const FwdParams& p, const LaunchShape& ls, cudaStream_t st);
-cudaError_t launch_updown(const FwdParams& p, int dtype, const LaunchShape& ls, cudaStream_t st);
-cudaError_t launch_finalize(const FwdParams& p, int dtype, const LaunchShape& ls, cudaStream_t st);
+int router_hsplit(int E, int B, int H);
+// pdl: launch with programmatic stream serialization (off while stage timing events are set)
+cudaError_t launch_gate(const FwdParams& p, int dtype, const LaunchShape& ls, cudaStream_t st,
+                        bool pdl);
+cudaError_t launch_select(const FwdParams& p, const LaunchShape& ls, cudaStream_t st, bool pdl);
+cudaError_t launch_updown(const FwdParams& p, int dtype, const LaunchShape& ls, cudaStream_t st,
+                          bool pdl);
+cudaError_t launch_finalize(const FwdParams& p, int dtype, const LaunchShape& ls, cudaStream_t st,
+                            bool pdl);
 
 // Set-up (called once per handle): shared-memory limits and persistent grid sizes.
-cudaError_t configure_kernels(int dtype, int imax, int max_E, int max_B, LaunchShape* ls);
+cudaError_t configure_kernels(int dtype, int imax, int max_E, int max_B, int H, LaunchShape* ls);
 size_t router_smem_bytes(int E, int B);
 size_t select_smem_bytes(int imax);
 

@@ -3,10 +3,10 @@
 
 namespace moe {
 
-int gate_occupancy(int dtype);
-int updown_occupancy(int dtype);
 cudaError_t configure_router(int max_E, int max_B);
 cudaError_t configure_select(int imax, int* occupancy);
+cudaError_t configure_gate(int dtype, int H, int smem_budget, LaunchShape* ls);
+cudaError_t configure_updown(int dtype, int H, int smem_budget, LaunchShape* ls);
 
 namespace {
 
@@ -14,7 +14,9 @@ namespace {
 template <typename T>
 __global__ void finalize_kernel(FwdParams p) {
   pdl_trigger();
+  trace_point(p.trace, 4, 0);
   pdl_wait();
+  trace_point(p.trace, 4, 1);
   const size_t n4 = (size_t)p.B * p.H / 4;
   float4* acc = reinterpret_cast<float4*>(p.out_acc);
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
@@ -68,15 +70,16 @@ __global__ void debug_gather_kernel(FwdParams p, int* cnt, int* lists, float* ac
 
 }  // namespace
 
-cudaError_t launch_finalize(const FwdParams& p, int dtype, const LaunchShape& ls, cudaStream_t st) {
+cudaError_t launch_finalize(const FwdParams& p, int dtype, const LaunchShape& ls, cudaStream_t st,
+                            bool pdl) {
   const size_t n4 = (size_t)p.B * p.H / 4;
   size_t blocks = (n4 + 255) / 256;
   const size_t cap = (size_t)ls.nsm * 4;
   if (blocks > cap) blocks = cap;
   if (dtype == 0)
     return launch_pdl(finalize_kernel<__nv_bfloat16>, dim3((unsigned)blocks), dim3(256), 0, st,
-                      true, p);
-  return launch_pdl(finalize_kernel<float>, dim3((unsigned)blocks), dim3(256), 0, st, true, p);
+                      pdl, p);
+  return launch_pdl(finalize_kernel<float>, dim3((unsigned)blocks), dim3(256), 0, st, pdl, p);
 }
 
 cudaError_t launch_pack_down(const void* w_down, void* packed_updown, int n, int I, int H,
@@ -98,22 +101,25 @@ cudaError_t launch_debug_gather(const FwdParams& p, int n_tokens, int* cnt, int*
   return cudaGetLastError();
 }
 
-cudaError_t configure_kernels(int dtype, int imax, int max_E, int max_B, LaunchShape* ls) {
+cudaError_t configure_kernels(int dtype, int imax, int max_E, int max_B, int H, LaunchShape* ls) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   e = cudaDeviceGetAttribute(&ls->nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  int budget = 0;
+  e = cudaDeviceGetAttribute(&budget, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (e != cudaSuccess) return e;
   e = configure_router(max_E, max_B);
   if (e != cudaSuccess) return e;
   int occ_sel = 0;
   e = configure_select(imax, &occ_sel);
   if (e != cudaSuccess) return e;
-  const int occ_gate = gate_occupancy(dtype);
-  const int occ_ud = updown_occupancy(dtype);
-  ls->grid_gate = ls->nsm * (occ_gate > 0 ? occ_gate : 1);
-  ls->grid_updown = ls->nsm * (occ_ud > 0 ? occ_ud : 1);
   ls->grid_select = ls->nsm * (occ_sel > 0 ? occ_sel : 1);
+  e = configure_gate(dtype, H, budget, ls);
+  if (e != cudaSuccess) return e;
+  e = configure_updown(dtype, H, budget, ls);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

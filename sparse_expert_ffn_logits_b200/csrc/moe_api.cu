@@ -11,6 +11,7 @@
 // Nothing is allocated and nothing waits on the host, so a call can be captured in a graph.
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <new>
@@ -36,6 +37,9 @@ struct moe_handle {
   void* out_stage;
   bool dirty;       // a call failed mid-way: re-zero before the next one
   int last_tokens;
+  cudaEvent_t stage_events[MOE_STAGE_EVENTS];
+  bool timing;
+  unsigned long long* trace_buf;  // device, kTraceKernels * kTraceCtas * kTracePoints stamps
 };
 
 namespace {
@@ -98,6 +102,7 @@ size_t carve(moe_handle* h, char* base) {
   Carve cv{base, 0};
   FwdParams& p = h->base;
   p.logits = cv.take<float>(Bm * E);
+  p.logit_part = cv.take<float>((size_t)moe::kMaxHsplit * Bm * E);
   p.topk_idx = cv.take<int>(Bm * k);
   p.topk_w = cv.take<float>(Bm * k);
   p.pair_index = cv.take<int>(Bm * (k + S));
@@ -113,6 +118,10 @@ size_t carve(moe_handle* h, char* base) {
   p.ulist = cv.take<int>(slots * Im);
   p.ucnt = cv.take<int>(slots);
   p.err = cv.take<int>(1);
+  p.zero_row = cv.take<char>((size_t)c.hidden * h->elt);
+  h->trace_buf = cv.take<unsigned long long>((size_t)moe::kTraceKernels * moe::kTraceCtas *
+                                             moe::kTracePoints);
+  p.trace = nullptr;
   h->x_stage = cv.take<char>(Bm * c.hidden * h->elt);
   h->out_stage = cv.take<char>(Bm * c.hidden * h->elt);
   // zero-at-rest region: tickets, union bitmasks, output accumulator
@@ -143,6 +152,8 @@ moe_status forward_impl(moe_handle* h, const void* x, int n_tokens, const void* 
   p.Ish = c.n_shared > 0 ? c.inter_shared : 0;
   p.B = n_tokens;
   p.Imax = h->imax;
+  p.Bmax = c.max_tokens;
+  p.hsplit = moe::router_hsplit(c.n_routed, n_tokens, c.hidden);
   p.route = (int)c.route;
   p.sel_mode[0] = sp_routed->mode == MOE_SEL_THRESHOLD ? 1 : 0;
   p.sel_K[0] = keep_count(c.inter, sp_routed->sparsity);
@@ -168,11 +179,23 @@ moe_status forward_impl(moe_handle* h, const void* x, int n_tokens, const void* 
     h->dirty = false;
   }
   const int dt = c.dtype == MOE_BF16 ? 0 : 1;
-  cudaError_t e = moe::launch_router(p, dt, st);
-  if (e == cudaSuccess) e = moe::launch_gate(p, dt, h->ls, st);
-  if (e == cudaSuccess) e = moe::launch_select(p, h->ls, st);
-  if (e == cudaSuccess) e = moe::launch_updown(p, dt, h->ls, st);
-  if (e == cudaSuccess) e = moe::launch_finalize(p, dt, h->ls, st);
+  // MOE_NO_PDL=1 in the environment launches the chain without programmatic overlap (a tuning
+  // switch; results are identical either way)
+  static const bool no_pdl = getenv("MOE_NO_PDL") != nullptr && getenv("MOE_NO_PDL")[0] == '1';
+  const bool tm = h->timing, pdl = !tm && !no_pdl;
+  p.trace = tm ? h->trace_buf : nullptr;
+  cudaEvent_t* ev = h->stage_events;
+  cudaError_t e = tm ? cudaEventRecord(ev[0], st) : cudaSuccess;
+  if (e == cudaSuccess) e = moe::launch_router(p, dt, st);
+  if (e == cudaSuccess && tm) e = cudaEventRecord(ev[1], st);
+  if (e == cudaSuccess) e = moe::launch_gate(p, dt, h->ls, st, pdl);
+  if (e == cudaSuccess && tm) e = cudaEventRecord(ev[2], st);
+  if (e == cudaSuccess) e = moe::launch_select(p, h->ls, st, pdl);
+  if (e == cudaSuccess && tm) e = cudaEventRecord(ev[3], st);
+  if (e == cudaSuccess) e = moe::launch_updown(p, dt, h->ls, st, pdl);
+  if (e == cudaSuccess && tm) e = cudaEventRecord(ev[4], st);
+  if (e == cudaSuccess) e = moe::launch_finalize(p, dt, h->ls, st, pdl);
+  if (e == cudaSuccess && tm) e = cudaEventRecord(ev[5], st);
   if (e != cudaSuccess) {
     h->dirty = true;
     return MOE_ERR_CUDA;
@@ -223,7 +246,7 @@ moe_status moe_create(const moe_config* cfg, moe_handle** out) {
     return MOE_ERR_CUDA;
   }
   cudaError_t e = moe::configure_kernels(cfg->dtype == MOE_BF16 ? 0 : 1, h->imax, cfg->n_routed,
-                                         cfg->max_tokens, &h->ls);
+                                         cfg->max_tokens, cfg->hidden, &h->ls);
   if (e != cudaSuccess) {
     delete h;
     return MOE_ERR_CUDA;
@@ -333,6 +356,33 @@ moe_status moe_debug_lists(moe_handle* h, int n_tokens, int* idx, float* w, floa
   if (e == cudaSuccess && (cnt || lists || act))
     e = moe::launch_debug_gather(p, n_tokens, cnt, lists, act, st);
   return cuda_status(e);
+}
+
+moe_status moe_profile_stages(moe_handle* h, void* const* events, int n_events) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (!events) {
+    h->timing = false;
+    return MOE_OK;
+  }
+  if (n_events != MOE_STAGE_EVENTS) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < MOE_STAGE_EVENTS; ++i) {
+    if (!events[i]) return MOE_ERR_INVALID_ARG;
+    h->stage_events[i] = static_cast<cudaEvent_t>(events[i]);
+  }
+  h->timing = true;
+  return MOE_OK;
+}
+
+moe_status moe_read_trace(moe_handle* h, unsigned long long* host, size_t n) {
+  if (!h || !host) return MOE_ERR_INVALID_ARG;
+  const size_t cap = (size_t)moe::kTraceKernels * moe::kTraceCtas * moe::kTracePoints;
+  if (n > cap) n = cap;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemcpy(host, h->trace_buf, n * sizeof(unsigned long long), cudaMemcpyDeviceToHost) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  return cudaMemset(h->trace_buf, 0, n * sizeof(unsigned long long)) == cudaSuccess ? MOE_OK
+                                                                                      : MOE_ERR_CUDA;
 }
 
 moe_status moe_get_error(moe_handle* h, int* device_code) {

@@ -19,149 +19,175 @@
 namespace moe {
 namespace {
 
-__device__ __forceinline__ bool better(float v, int e, float bv, int be) {
-  return v > bv || (v == bv && e < be);
+// Order key of (logit, expert): larger key = larger logit, then lower expert index; 0 = none.
+__device__ __forceinline__ unsigned long long topk_key(float v, int e) {
+  uint32_t u = __float_as_uint(v);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ((unsigned long long)u << 32) | (0xFFFFFFFFu - (uint32_t)e);
+}
+__device__ __forceinline__ float key_value(unsigned long long k) {
+  uint32_t u = (uint32_t)(k >> 32);
+  u = (u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u;
+  return __uint_as_float(u);
 }
 
-// Top-k of one token's logits by one warp; writes topk_idx / topk_w.
-__device__ void topk_token(const FwdParams& p, int tok) {
+// Top-k of one token's logits (lg, shared memory) by one warp; writes topk_idx / topk_w.
+// PER = logits per lane (E <= 32 * PER).  sv / si: this warp's k-entry scratch.
+template <int PER>
+__device__ void topk_token(const FwdParams& p, int tok, const float* lg, float* sv, int* si) {
   const int lane = threadIdx.x & 31;
   const int E = p.E, k = p.k;
-  constexpr int kPer = kMaxRouted / 32;
-  float v[kPer];
+  unsigned long long key[PER];
   bool nan_seen = false;
 #pragma unroll
-  for (int j = 0; j < kPer; ++j) {
+  for (int j = 0; j < PER; ++j) {
     const int e = lane + 32 * j;
-    float f = -INFINITY;
+    key[j] = 0ull;
     if (e < E) {
-      f = ld_cg(&p.logits[(size_t)tok * E + e]);
+      float f = lg[e];
       if (isnan(f)) {
         nan_seen = true;
         f = -INFINITY;
       }
+      key[j] = topk_key(f, e);
     }
-    v[j] = f;
   }
   if (__any_sync(0xffffffffu, nan_seen) && lane == 0) set_error(p.err, kErrNanLogit);
-  unsigned taken = 0;
-  float sel_v[kMaxTopK];
-  int sel_e[kMaxTopK];
+  for (int r = 0; r < k; ++r) {
+    unsigned long long best = key[0];
 #pragma unroll
-  for (int r = 0; r < kMaxTopK; ++r) {
-    sel_v[r] = -INFINITY;
-    sel_e[r] = 0;
-    if (r < k) {
-      float bv = -INFINITY;
-      int be = 0x7fffffff;
+    for (int j = 1; j < PER; ++j) best = key[j] > best ? key[j] : best;
 #pragma unroll
-      for (int j = 0; j < kPer; ++j) {
-        const int e = lane + 32 * j;
-        if (e < E && !((taken >> j) & 1u) && better(v[j], e, bv, be)) {
-          bv = v[j];
-          be = e;
-        }
-      }
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+      best = other > best ? other : best;
+    }
+    const int e = (int)(0xFFFFFFFFu - (uint32_t)best);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-        if (better(ov, oe, bv, be)) {
-          bv = ov;
-          be = oe;
-        }
-      }
-      if ((be & 31) == lane) taken |= 1u << (be >> 5);
-      sel_v[r] = bv;
-      sel_e[r] = be;
+    for (int j = 0; j < PER; ++j)
+      if (lane + 32 * j == e) key[j] = 0ull;
+    if (lane == 0) {
+      si[r] = e;
+      sv[r] = key_value(best);
     }
   }
-  float w[kMaxTopK];
-  if (p.route == 2) {
+  __syncwarp();
+  // routing weights: lane r < k computes entry r
+  float z = 0.f;
+  const float m = sv[0];
+  if (p.route == 1) {
 #pragma unroll
-    for (int r = 0; r < kMaxTopK; ++r) w[r] = 1.0f / (1.0f + expf(-sel_v[r]));
-  } else {
-    const float m = sel_v[0];
-    float z = 0.f;
-    if (p.route == 1) {
-#pragma unroll
-      for (int j = 0; j < kPer; ++j)
-        if (lane + 32 * j < E) z += expf(v[j] - m);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-    } else {
-#pragma unroll
-      for (int r = 0; r < kMaxTopK; ++r)
-        if (r < k) z += expf(sel_v[r] - m);
+    for (int j = 0; j < PER; ++j) {
+      const int e = lane + 32 * j;
+      if (e < E) {
+        const float f = lg[e];
+        z += expf((isnan(f) ? -INFINITY : f) - m);
+      }
     }
 #pragma unroll
-    for (int r = 0; r < kMaxTopK; ++r) w[r] = expf(sel_v[r] - m) / z;
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+  } else if (p.route == 0) {
+    for (int r = 0; r < k; ++r) z += expf(sv[r] - m);
   }
-#pragma unroll
-  for (int r = 0; r < kMaxTopK; ++r) {
-    if (r < k && lane == r) {
-      p.topk_idx[(size_t)tok * k + r] = sel_e[r];
-      p.topk_w[(size_t)tok * k + r] = w[r];
-    }
+  if (lane < k) {
+    const float v = sv[lane];
+    const float w = p.route == 2 ? 1.0f / (1.0f + expf(-v)) : expf(v - m) / z;
+    p.topk_idx[(size_t)tok * k + lane] = si[lane];
+    p.topk_w[(size_t)tok * k + lane] = w;
   }
 }
 
-// Exclusive scan of n ints in place (shared memory), by the whole block; returns the total.
-__device__ int block_scan_array(int* a, int n, int* scratch) {
-  const int per = (n + blockDim.x - 1) / blockDim.x;
-  const int beg = min(n, (int)threadIdx.x * per), end = min(n, beg + per);
-  int s = 0;
-  for (int i = beg; i < end; ++i) s += a[i];
-  int total;
-  int run = block_exclusive_scan(s, scratch, &total);
-  for (int i = beg; i < end; ++i) {
-    const int v = a[i];
-    a[i] = run;
-    run += v;
+// Exclusive prefix of a 64-bit value over the block; scratch holds 33 x 64 bits.
+__device__ unsigned long long block_scan64(unsigned long long v, unsigned long long* scratch,
+                                           unsigned long long* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  unsigned long long incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) scratch[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const unsigned long long s = lane < nw ? scratch[lane] : 0ull;
+    unsigned long long si = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned long long y = __shfl_up_sync(0xffffffffu, si, o);
+      if (lane >= o) si += y;
+    }
+    if (lane < nw) scratch[lane] = si - s;
+    if (lane == 31) scratch[32] = si;
   }
   __syncthreads();
-  return total;
+  const unsigned long long res = scratch[warp] + incl - v;
+  *total = scratch[32];
+  __syncthreads();
+  return res;
 }
 
-// Groups all pairs by expert and writes the slot table, pair arrays and meta (one CTA).
-__device__ void group_pairs(const FwdParams& p, uint32_t* dyn, int* scratch) {
+// Groups all pairs by expert (tokens ascending within an expert) and writes the slot table,
+// the pair arrays and meta (one CTA).  One 64-bit block scan over the experts gives, packed,
+// each expert's first pair, its slot index and its first gate item.
+__device__ void group_pairs(const FwdParams& p, uint32_t* dyn, unsigned long long* scratch) {
   const int B = p.B, E = p.E, k = p.k, S = p.S;
   const int W = (B + 31) / 32;
-  int* cnt = reinterpret_cast<int*>(dyn);  // [E]
-  int* qoff = cnt + E;                     // [E] exclusive prefix of cnt
-  int* touched = qoff + E;                 // [E] -> slot index after the scan
-  int* items = touched + E;                // [E + S] gate items per slot -> item0
-  uint32_t* tokmask = reinterpret_cast<uint32_t*>(items + E + S);  // [E][W]
+  int* cnt = reinterpret_cast<int*>(dyn);                          // [E]
+  unsigned long long* pre = reinterpret_cast<unsigned long long*>(
+      dyn + ((E + 1) & ~1));                                      // [E] packed prefixes
+  uint32_t* tokmask = reinterpret_cast<uint32_t*>(pre + E);        // [E][W]
+  int* sidx = reinterpret_cast<int*>(tokmask + E * W);             // [B*k]
+  float* sw = reinterpret_cast<float*>(sidx + B * k);              // [B*k]
   for (int i = threadIdx.x; i < E; i += blockDim.x) cnt[i] = 0;
   for (int i = threadIdx.x; i < E * W; i += blockDim.x) tokmask[i] = 0;
+  for (int i = threadIdx.x; i < B * k; i += blockDim.x) {
+    sidx[i] = ld_cg(&p.topk_idx[i]);
+    sw[i] = ld_cg(&p.topk_w[i]);
+  }
   __syncthreads();
   for (int pi = threadIdx.x; pi < B * k; pi += blockDim.x) {
-    const int t = pi / k;
-    const int e = ld_cg(&p.topk_idx[pi]);
+    const int t = pi / k, e = sidx[pi];
     atomicAdd(&cnt[e], 1);
     atomicOr(&tokmask[e * W + (t >> 5)], 1u << (t & 31));
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    qoff[e] = cnt[e];
-    touched[e] = cnt[e] > 0 ? 1 : 0;
+  // packed per expert: pairs (bits 0..19) | touched (bits 20..31) | gate items (bits 32..63)
+  const int per = (E + blockDim.x - 1) / blockDim.x;
+  const int e0 = min(E, (int)threadIdx.x * per), e1 = min(E, e0 + per);
+  unsigned long long mine = 0ull;
+  for (int e = e0; e < e1; ++e) {
+    const unsigned long long c = (unsigned)cnt[e];
+    const unsigned long long items =
+        c ? (unsigned long long)(p.I / kTileRows) * ((c + kTileTok - 1) / kTileTok) : 0ull;
+    mine += c | ((c ? 1ull : 0ull) << 20) | (items << 32);
+  }
+  unsigned long long tot;
+  unsigned long long run = block_scan64(mine, scratch, &tot);
+  for (int e = e0; e < e1; ++e) {
+    pre[e] = run;
+    const unsigned long long c = (unsigned)cnt[e];
+    run += c | ((c ? 1ull : 0ull) << 20) |
+           ((c ? (unsigned long long)(p.I / kTileRows) * ((c + kTileTok - 1) / kTileTok) : 0ull)
+            << 32);
   }
   __syncthreads();
-  block_scan_array(qoff, E, scratch);
-  const int n_touched = block_scan_array(touched, E, scratch);
+  const int n_touched = (int)((tot >> 20) & 0xFFF);
+  const int routed_items = (int)(tot >> 32);
   const int n_slots = n_touched + S;
+  const int sh_items = (p.Ish / kTileRows) * ((B + kTileTok - 1) / kTileTok);
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     if (cnt[e] > 0) {
+      const unsigned long long pr = pre[e];
       Slot s;
       s.kind = 0;
       s.expert = e;
       s.T = cnt[e];
-      s.q0 = qoff[e];
+      s.q0 = (int)(pr & 0xFFFFF);
       s.I = p.I;
-      s.item0 = 0;
+      s.item0 = (int)(pr >> 32);
       s.pad0 = s.pad1 = 0;
-      p.slots[touched[e]] = s;
-      items[touched[e]] = (p.I / kTileRows) * ((cnt[e] + kTileTok - 1) / kTileTok);
+      p.slots[(int)((pr >> 20) & 0xFFF)] = s;
     }
   }
   for (int s_i = threadIdx.x; s_i < S; s_i += blockDim.x) {
@@ -171,21 +197,20 @@ __device__ void group_pairs(const FwdParams& p, uint32_t* dyn, int* scratch) {
     s.T = B;
     s.q0 = B * k + s_i * B;
     s.I = p.Ish;
-    s.item0 = 0;
+    s.item0 = routed_items + s_i * sh_items;
     s.pad0 = s.pad1 = 0;
     p.slots[n_touched + s_i] = s;
-    items[n_touched + s_i] = (p.Ish / kTileRows) * ((B + kTileTok - 1) / kTileTok);
   }
   // routed pairs: rank of token t among the tokens of its expert
   for (int pi = threadIdx.x; pi < B * k; pi += blockDim.x) {
-    const int t = pi / k;
-    const int e = ld_cg(&p.topk_idx[pi]);
+    const int t = pi / k, e = sidx[pi];
     int rank = __popc(tokmask[e * W + (t >> 5)] & ((1u << (t & 31)) - 1u));
     for (int w = 0; w < (t >> 5); ++w) rank += __popc(tokmask[e * W + w]);
-    const int q = qoff[e] + rank;
+    const unsigned long long pr = pre[e];
+    const int q = (int)(pr & 0xFFFFF) + rank;
     p.pair_token[q] = t;
-    p.pair_w[q] = ld_cg(&p.topk_w[pi]);
-    p.pair_slot[q] = touched[e];
+    p.pair_w[q] = sw[pi];
+    p.pair_slot[q] = (int)((pr >> 20) & 0xFFF);
     p.pair_index[t * (k + S) + (pi % k)] = q;
   }
   for (int i = threadIdx.x; i < B * S; i += blockDim.x) {
@@ -196,28 +221,35 @@ __device__ void group_pairs(const FwdParams& p, uint32_t* dyn, int* scratch) {
     p.pair_slot[q] = n_touched + s_i;
     p.pair_index[t * (k + S) + k + s_i] = q;
   }
-  __syncthreads();
-  const int n_items = block_scan_array(items, n_slots, scratch);
-  for (int j = threadIdx.x; j < n_slots; j += blockDim.x) p.slots[j].item0 = items[j];
   if (threadIdx.x == 0) {
     p.meta[kMetaSlots] = n_slots;
     p.meta[kMetaPairs] = B * (k + S);
-    p.meta[kMetaGateItems] = n_items;
+    p.meta[kMetaGateItems] = routed_items + S * sh_items;
     p.meta[kMetaTouched] = n_touched;
   }
 }
 
-template <typename T>
+// Grid (egroups * hsplit, token tiles).  CTA (eg, hs, tt): partial logits of experts 16eg..
+// over the hs-th slice of H for the 8 tokens of tile tt; the last CTA of the tile (ticket) sums
+// the slices in a fixed order, picks the top-k, and the last tile groups the pairs.
+template <typename T, int PER>
 __global__ void __launch_bounds__(kThreads) router_kernel(FwdParams p) {
   __shared__ float red[kWarps][32][4];
   __shared__ const T* s_x[kTileTok];
   __shared__ int s_last;
-  __shared__ int scratch[33];
+  __shared__ unsigned long long scratch[33];
+  __shared__ float s_lg[kTileTok][kMaxRouted];
+  __shared__ float s_tv[kWarps][kMaxTopK];
+  __shared__ int s_ti[kWarps][kMaxTopK];
   extern __shared__ uint32_t dyn[];
   pdl_trigger();
+  trace_point(p.trace, 0, 0);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
-  const int H = p.H, E = p.E, B = p.B;
-  const int e0 = blockIdx.x * kTileRows, tt = blockIdx.y;
+  const int H = p.H, E = p.E, B = p.B, hsplit = p.hsplit;
+  const int eg = blockIdx.x / hsplit, hs = blockIdx.x % hsplit, tt = blockIdx.y;
+  const int e0 = eg * kTileRows;
+  const int nblk = H / 32;
+  const int blo = hs * nblk / hsplit, bhi = (hs + 1) * nblk / hsplit;
   const T* x = static_cast<const T*>(p.x);
   const T* wr = static_cast<const T*>(p.router);
   if (threadIdx.x < kTileTok) {
@@ -228,26 +260,23 @@ __global__ void __launch_bounds__(kThreads) router_kernel(FwdParams p) {
   const T* rowA = wr + (size_t)min(e0 + g, E - 1) * H;
   const T* rowB = wr + (size_t)min(e0 + g + 8, E - 1) * H;
   float d[4] = {0.f, 0.f, 0.f, 0.f};
-  tile_dot<2>(rowA, rowB, s_x, warp, kWarps, H / 32, d);
+  tile_dot<4>(rowA, rowB, s_x, blo + warp, kWarps, bhi, d);
 #pragma unroll
   for (int c = 0; c < 4; ++c) red[warp][lane][c] = d[c];
   __syncthreads();
   if (warp == 0) {
     reduce_fragments(red, d);
-    bool nan_seen = false;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       const int e = e0 + g + (c >> 1) * 8;
       const int tok = tt * kTileTok + 2 * t + (c & 1);
-      if (e < E && tok < B) {
-        p.logits[(size_t)tok * E + e] = d[c];
-        nan_seen |= isnan(d[c]);
-      }
+      if (e < E && tok < B) p.logit_part[((size_t)hs * p.Bmax + tok) * E + e] = d[c];
     }
-    if (nan_seen) set_error(p.err, kErrNanLogit);
   }
+  trace_point(p.trace, 0, 1);
   __threadfence();
   __syncthreads();
+  trace_point(p.trace, 0, 2);
   if (threadIdx.x == 0) {
     const unsigned ticket = atomicAdd(&p.tile_ticket[tt], 1u);
     s_last = ticket == gridDim.x - 1;
@@ -255,10 +284,31 @@ __global__ void __launch_bounds__(kThreads) router_kernel(FwdParams p) {
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  // logits of the tile's tokens: the H slices summed in a fixed order
+  bool nan_seen = false;
+  for (int i = threadIdx.x; i < kTileTok * E; i += blockDim.x) {
+    const int c = i / E, e = i % E, tok = tt * kTileTok + c;
+    float v = 0.f;
+    if (tok < B) {
+      float pv[kMaxHsplit];  // all slices in flight at once, then summed in slice order
+#pragma unroll
+      for (int h = 0; h < kMaxHsplit; ++h)
+        pv[h] = h < hsplit ? ld_cg(&p.logit_part[((size_t)h * p.Bmax + tok) * E + e]) : 0.f;
+#pragma unroll
+      for (int h = 0; h < kMaxHsplit; ++h) v += pv[h];
+      p.logits[(size_t)tok * E + e] = v;
+      nan_seen |= isnan(v);
+    }
+    s_lg[c][e] = v;
+  }
+  if (nan_seen) set_error(p.err, kErrNanLogit);
+  __syncthreads();
+  trace_point(p.trace, 0, 3);
   {
     const int tok = tt * kTileTok + warp;
-    if (tok < B) topk_token(p, tok);
+    if (tok < B) topk_token<PER>(p, tok, s_lg[warp], s_tv[warp], s_ti[warp]);
   }
+  trace_point(p.trace, 0, 4);
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -269,32 +319,67 @@ __global__ void __launch_bounds__(kThreads) router_kernel(FwdParams p) {
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  trace_point(p.trace, 0, 5);
   group_pairs(p, dyn, scratch);
   if (threadIdx.x == 0) *p.global_ticket = 0;
+  trace_point(p.trace, 0, 6);
 }
 
 }  // namespace
 
 size_t router_smem_bytes(int E, int B) {
   const int W = (B + 31) / 32;
-  return sizeof(int) * (size_t)(3 * E + E + kMaxShared) + sizeof(uint32_t) * (size_t)E * W;
+  // cnt [E] (padded to even) | packed prefixes [E] x 8 | tokmask [E][W] | topk idx, w [B*k]
+  return sizeof(int) * (size_t)((E + 1) & ~1) + 8 * (size_t)E + 4 * (size_t)E * W +
+         (size_t)B * kMaxTopK * 8;
+}
+
+// H slices of the router: enough CTAs to keep ~96 in flight, at least 2 blocks of 32 per slice.
+int router_hsplit(int E, int B, int H) {
+  const int ctas = ((E + kTileRows - 1) / kTileRows) * ((B + kTileTok - 1) / kTileTok);
+  int hs = (96 + ctas - 1) / ctas;
+  const int cap = H / 64;
+  if (hs > cap) hs = cap;
+  if (hs > kMaxHsplit) hs = kMaxHsplit;
+  return hs < 1 ? 1 : hs;
+}
+
+template <typename T>
+cudaError_t launch_router_t(const FwdParams& p, dim3 grid, size_t smem, cudaStream_t st) {
+  if (p.E <= 32) return launch_pdl(router_kernel<T, 1>, grid, dim3(kThreads), smem, st, false, p);
+  if (p.E <= 64) return launch_pdl(router_kernel<T, 2>, grid, dim3(kThreads), smem, st, false, p);
+  if (p.E <= 128) return launch_pdl(router_kernel<T, 4>, grid, dim3(kThreads), smem, st, false, p);
+  if (p.E <= 256) return launch_pdl(router_kernel<T, 8>, grid, dim3(kThreads), smem, st, false, p);
+  return launch_pdl(router_kernel<T, 16>, grid, dim3(kThreads), smem, st, false, p);
 }
 
 cudaError_t launch_router(const FwdParams& p, int dtype, cudaStream_t st) {
-  dim3 grid((p.E + kTileRows - 1) / kTileRows, (p.B + kTileTok - 1) / kTileTok);
+  dim3 grid(((p.E + kTileRows - 1) / kTileRows) * p.hsplit, (p.B + kTileTok - 1) / kTileTok);
   const size_t smem = router_smem_bytes(p.E, p.B);
-  if (dtype == 0)
-    return launch_pdl(router_kernel<__nv_bfloat16>, grid, dim3(kThreads), smem, st, false, p);
-  return launch_pdl(router_kernel<float>, grid, dim3(kThreads), smem, st, false, p);
+  if (dtype == 0) return launch_router_t<__nv_bfloat16>(p, grid, smem, st);
+  return launch_router_t<float>(p, grid, smem, st);
+}
+
+template <typename T>
+cudaError_t configure_router_t(int smem) {
+  cudaError_t e = cudaSuccess;
+  e = cudaFuncSetAttribute(router_kernel<T, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(router_kernel<T, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(router_kernel<T, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(router_kernel<T, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(router_kernel<T, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  return e;
 }
 
 cudaError_t configure_router(int max_E, int max_B) {
-  const size_t smem = router_smem_bytes(max_E, max_B);
-  cudaError_t e = cudaFuncSetAttribute(router_kernel<__nv_bfloat16>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const int smem = (int)router_smem_bytes(max_E, max_B);
+  cudaError_t e = configure_router_t<__nv_bfloat16>(smem);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(router_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)smem);
+  return configure_router_t<float>(smem);
 }
 
 }  // namespace moe

@@ -3,14 +3,16 @@
 // Inside a pair the lowest-scoring neuron activations are dropped ("Uncovering Intra-expert
 // Activation Sparsity ...", technical summary, Methodology: activation masking).  The score of
 // neuron n is |SiLU(g_n)|, an fp32 value whose bit pattern (sign cleared) orders like the value.
-//   top-K mode: an MSB-first radix select (four 8-bit digits, shared-memory histograms) finds
-//     the K-th largest key tau and how many keys equal to tau are kept; the kept set is every
-//     key > tau plus the lowest-indexed keys == tau.  No sort.
+//   top-K mode: an MSB-first radix select (four 8-bit digits) finds the K-th largest key tau
+//     and how many keys equal to tau are kept; the kept set is every key > tau plus the
+//     lowest-indexed keys == tau.  No sort.
 //   threshold mode: one pass, keep key > t (the page's single-pass threshold mask).
-// The kept set is written as an ascending index list + count (for export), as a bitmask row,
-// and OR-ed into the expert's union bitmask.  The last pair of an expert to finish (atomic
-// ticket, no waiting) compacts the union into an ascending row list for the up/down kernel and
-// clears the bitmask for the next call.
+// One CTA per pair: its keys sit in shared memory; each warp histograms its share of them into
+// its own 256 bins (lanes holding the same digit are merged by a match-any vote, one plain add
+// per distinct digit), and a block scan over the summed bins finds the digit.  The kept set is
+// written as an ascending index list + count (for export), as a bitmask row, and OR-ed into the
+// expert's union bitmask.  The last pair of an expert to finish (atomic ticket, no waiting)
+// compacts the union into an ascending row list for the up/down kernel and clears the bitmask.
 #include "kernels.h"
 
 namespace moe {
@@ -21,79 +23,88 @@ constexpr int kSelWarps = kSelThreads / 32;
 
 __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
   extern __shared__ uint32_t sm[];
-  __shared__ int hist[256];
+  __shared__ int hist[kSelWarps][256];
   __shared__ int scratch[33];
   __shared__ int wtot[kSelWarps];
   __shared__ int s_digit, s_above, s_last;
   pdl_trigger();
+  trace_point(p.trace, 2, 0);
   pdl_wait();
+  trace_point(p.trace, 2, 1);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int Imax = p.Imax, Wmax = p.Imax / 32;
-  uint32_t* key = sm;                                               // [Imax]
+  uint32_t* key = sm;                                                 // [Imax]
   unsigned char* keep = reinterpret_cast<unsigned char*>(sm + Imax);  // [Imax]
   const int n_pairs = ld_cg(&p.meta[kMetaPairs]);
   bool nan_seen = false;
   for (int q = blockIdx.x; q < n_pairs; q += gridDim.x) {
-    const int j = p.pair_slot[q];
-    const Slot s = p.slots[j];
+    const int j = __ldcg(&p.pair_slot[q]);
+    const Slot s = load_slot(&p.slots[j]);
     const int I = s.I, kind = s.kind;
-    const float* a = p.act + (size_t)q * Imax;
-    for (int n = threadIdx.x; n < I; n += blockDim.x) {
-      const float f = a[n];
-      uint32_t u = __float_as_uint(fabsf(f));
-      if (isnan(f)) {
-        nan_seen = true;
-        u = 0;
+    {
+      const float4* a4 = reinterpret_cast<const float4*>(p.act + (size_t)q * Imax);
+      for (int v0 = threadIdx.x; v0 < I / 4; v0 += 4 * kSelThreads) {
+        float4 f[4];  // four 16-byte loads in flight per thread
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          f[u] = v0 + u * kSelThreads < I / 4 ? __ldcg(a4 + v0 + u * kSelThreads)
+                                              : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int v = v0 + u * kSelThreads;
+          if (v < I / 4) {
+            const float fv[4] = {f[u].x, f[u].y, f[u].z, f[u].w};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t k4 = __float_as_uint(fabsf(fv[c]));
+              if (isnan(fv[c])) {
+                nan_seen = true;
+                k4 = 0;
+              }
+              key[v * 4 + c] = k4;
+            }
+          }
+        }
       }
-      key[n] = u;
     }
     __syncthreads();
     const int mode = p.sel_mode[kind];
     const int K = min(p.sel_K[kind], I);
     const float thr = p.sel_t[kind];
+    const bool radix = mode == 0 && K > 0 && K < I;
     uint32_t tau = 0;
     int need = 0;
-    if (mode == 0 && K > 0 && K < I) {
+    if (radix) {
       uint32_t prefix = 0, pmask = 0;
       int krem = K;
       for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
-        __syncthreads();
-        for (int n = threadIdx.x; n < I; n += blockDim.x) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) hist[warp][lane * 8 + i] = 0;
+        __syncwarp();
+        for (int n = warp * 32 + lane; n < I; n += kSelThreads) {
           const uint32_t u = key[n];
-          if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1);
+          const bool match = (u & pmask) == prefix;
+          const uint32_t dg = match ? (u >> shift) & 255u : 256u + lane;
+          const unsigned same = __match_any_sync(0xffffffffu, dg);
+          if (match && lane == __ffs(same) - 1) hist[warp][dg] += __popc(same);
+          __syncwarp();
         }
         __syncthreads();
-        if (warp == 0) {
-          // lane l owns digits 255-8l .. 248-8l (descending); find the digit holding the
-          // krem-th largest key
-          int c[8], sum = 0;
+        // thread b holds digit 255 - b (descending order), summed over the warps
+        const int dig = 255 - (int)threadIdx.x;
+        int c = 0;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            c[i] = hist[255 - 8 * lane - i];
-            sum += c[i];
-          }
-          int incl = sum;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
-          }
-          int above = incl - sum;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            if (above < krem && above + c[i] >= krem) {
-              s_digit = 255 - 8 * lane - i;
-              s_above = above;
-            }
-            above += c[i];
-          }
+        for (int w = 0; w < kSelWarps; ++w) c += hist[w][dig];
+        int total;
+        const int above = block_exclusive_scan(c, scratch, &total);
+        if (above < krem && above + c >= krem) {
+          s_digit = dig;
+          s_above = above;
         }
         __syncthreads();
         krem -= s_above;
         prefix |= (uint32_t)s_digit << shift;
         pmask |= 255u << shift;
-        __syncthreads();
       }
       tau = prefix;
       need = krem;
@@ -102,7 +113,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
     const int seg = ((I + 32 * kSelWarps - 1) / (32 * kSelWarps)) * 32;
     const int sb = warp * seg, se = min(I, sb + seg);
     int tie_base = 0;
-    if (mode == 0 && K > 0 && K < I) {
+    if (radix) {
       int ties = 0;
       for (int n0 = sb; n0 < se; n0 += 32) {
         const int n = n0 + lane;
@@ -118,24 +129,21 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
       int run = tie_base;
       for (int n0 = sb; n0 < se; n0 += 32) {
         const int n = n0 + lane;
-        bool k_n = false;
-        if (n < se) {
-          const uint32_t u = key[n];
-          if (mode == 1) {
-            k_n = __uint_as_float(u) > thr;
-          } else if (K >= I) {
-            k_n = true;
-          } else if (K > 0) {
-            k_n = u > tau;
-          }
-        }
-        if (mode == 0 && K > 0 && K < I) {
-          const bool eq = n < se && key[n] == tau;
+        const uint32_t u = n < se ? key[n] : 0u;
+        bool k_n;
+        if (mode == 1) {
+          k_n = __uint_as_float(u) > thr;
+        } else if (K >= I) {
+          k_n = true;
+        } else if (K == 0) {
+          k_n = false;
+        } else {
+          const bool eq = n < se && u == tau;
           const unsigned be = __ballot_sync(0xffffffffu, eq);
-          const int rank = run + __popc(be & lanemask_lt());
-          if (eq && rank < need) k_n = true;
+          k_n = u > tau || (eq && run + __popc(be & lanemask_lt()) < need);
           run += __popc(be);
         }
+        k_n = k_n && n < se;
         if (n < se) keep[n] = k_n ? 1 : 0;
         kept += __popc(__ballot_sync(0xffffffffu, k_n));
       }
@@ -170,15 +178,15 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
     }
     __syncthreads();
     if (s_last) {
+      // last pair of this expert: compact the union bitmask into a row list, clear it
       __threadfence();
-      // compact the expert's union bitmask into an ascending row list, then clear it
       const int W = I / 32;
       const int per = (W + blockDim.x - 1) / blockDim.x;
       const int wb = min(W, (int)threadIdx.x * per), we = min(W, wb + per);
-      uint32_t words[4];
+      uint32_t words[2];
       int c = 0;
       for (int w = wb; w < we; ++w) {
-        words[w - wb] = ld_cg(&urow[w]);
+        words[w - wb] = __ldcg(&urow[w]);
         c += __popc(words[w - wb]);
       }
       int utotal;
@@ -187,8 +195,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
       for (int w = wb; w < we; ++w) {
         uint32_t b = words[w - wb];
         while (b) {
-          const int bit = __ffs(b) - 1;
-          ul[upos++] = w * 32 + bit;
+          ul[upos++] = w * 32 + __ffs(b) - 1;
           b &= b - 1;
         }
         urow[w] = 0;
@@ -201,17 +208,18 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
     __syncthreads();
   }
   if (nan_seen) set_error(p.err, kErrNanAct);
+  trace_point(p.trace, 2, 7);
 }
 
 }  // namespace
 
 size_t select_smem_bytes(int imax) { return (size_t)imax * 5 + 16; }
 
-cudaError_t launch_select(const FwdParams& p, const LaunchShape& ls, cudaStream_t st) {
+cudaError_t launch_select(const FwdParams& p, const LaunchShape& ls, cudaStream_t st, bool pdl) {
   const int pairs = p.B * (p.k + p.S);
   const int grid = pairs < ls.grid_select ? pairs : ls.grid_select;
   return launch_pdl(select_kernel, dim3(grid), dim3(kSelThreads), select_smem_bytes(p.Imax), st,
-                    true, p);
+                    pdl, p);
 }
 
 cudaError_t configure_select(int imax, int* occupancy) {

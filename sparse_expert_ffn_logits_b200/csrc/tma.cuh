@@ -1,0 +1,155 @@
+// tma.cuh - bulk asynchronous copies (TMA, non-tensor form) into a shared-memory ring with
+// mbarrier completion, and bounded waits.
+//
+// Only the plain single-CTA form is used: cp.async.bulk global -> shared of this CTA, completed
+// on an mbarrier by byte count.  Every wait is bounded by %globaltimer; on time-out the waiter
+// sets the device error word and a CTA-wide abort flag, after which no thread of the CTA waits
+// again, so the CTA always drains and exits.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kErrTimeout = 3;
+constexpr unsigned long long kWaitLimitNs = 200ull * 1000ull * 1000ull;  // 0.2 s
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+// Makes barrier initialisation visible to the async (copy) proxy; follow with __syncthreads.
+__device__ __forceinline__ void mbar_init_fence() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Waits for the phase of `bar` with parity `parity`.  Returns false (without waiting) once
+// *abort is set; on time-out sets *abort and the error word.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          int* err) {
+  if (mbar_test(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  while (true) {
+    if (*abort) return false;
+    if (mbar_test(bar, parity)) return true;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      *abort = 1;
+      set_error(err, kErrTimeout);
+      return false;
+    }
+  }
+}
+
+// Waits, bounded by time only (it ignores the abort flag), until a stage's copies have landed;
+// used before a producer exits so that no copy still targets the CTA's shared memory.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const unsigned long long t0 = globaltimer();
+  while (!mbar_test(bar, parity) && globaltimer() - t0 < kWaitLimitNs) {
+  }
+}
+
+// 1-D bulk copy global -> shared of this CTA, completing `bytes` on `bar`.  dst, src and bytes
+// must be multiples of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// 16-byte asynchronous copy global -> shared (L2 only), tracked per thread.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+// Arrives on `bar` once every cp.async this thread issued so far has landed; the arrival counts
+// against the barrier's expected count.
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(const void* p) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(smem_u32(p)));
+  return v;
+}
+
+// Named barrier over the first `n` threads of the CTA (the consumer warps).
+__device__ __forceinline__ void consumer_sync(int n) {
+  asm volatile("bar.sync 1, %0;" ::"r"(n) : "memory");
+}
+
+// Named barrier over the first `n` threads that also ORs `pred` across them: every participant
+// gets the same answer (used to take the abort decision uniformly).
+__device__ __forceinline__ int consumer_sync_or(int n, int pred) {
+  int r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.s32 p, %1, 0;\n bar.red.or.pred q, 1, %2, p;\n"
+      " selp.s32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"(pred), "r"(n)
+      : "memory");
+  return r;
+}
+
+// Shape of the copy ring of the gate and up/down kernels.
+struct Ring {
+  int ns;          // weight stages
+  int kc;          // h per stage (a multiple of 64 that divides H)
+  int nk;          // stages per row piece = H / kc
+  int stage_bytes; // bytes of one stage slot
+  int rs_a;        // row stride of stages read as "rows x h" (gate, up): kc*2 + 64
+  int rs_d;        // row stride of down stages: kc*2 + 16
+  int nxb;         // token tile buffers (2 when they fit)
+  int xs_stride;   // token row stride in a token tile: H*2 + 64
+  int xs_bytes;    // one token tile: 8 * xs_stride
+  int smem_bytes;  // dynamic shared memory of the kernel
+};
+
+// Dynamic shared memory of the ring kernels: barriers | 2 reduction tiles | token tiles | stages
+constexpr int kBarBytes = 512;
+constexpr int kRedBytes = 2 * 8 * 32 * 16;
+constexpr int kMetaRing = 4;
+
+
+}  // namespace moe

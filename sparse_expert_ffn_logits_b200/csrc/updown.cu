@@ -3,135 +3,428 @@
 // Only the weights of active neurons are read ("Uncovering Intra-expert Activation Sparsity
 // ...", technical summary, Methodology: fused up-down projection).  The packed layout keeps a
 // neuron's W_up row and W_down column side by side ([I][2][H]), so the rows of the expert's
-// kept-neuron union are gathered as contiguous 2*H*elt chunks and a dropped neuron costs no
-// bytes.  Each row is read once per token tile of its expert; tokens of the tile whose own
-// kept set lacks the neuron get coefficient 0.
+// kept-neuron union are gathered as contiguous pieces and a dropped neuron costs no bytes.
+// Each row is read once per token tile of its expert; tokens of the tile whose own kept set
+// lacks the neuron get coefficient 0.
 //
-// Work item = (slot, 16 union rows, token tile of 8 pairs), row group outer.  Per item:
-//   1. u[r][c] = W_up[n_r] . x_c           tensor cores, the 8 warps split H (tile_dot)
+// Work item = (slot, token tile of 8 pairs, 16 union rows), ordered slot, token tile, rows;
+// each CTA takes a contiguous range of items.  Per item:
+//   1. u[r][c] = W_up[n_r] . x_c           tensor cores, warps split H
 //   2. hc[r][c] = mask * SiLU(g) * u        fp32, rounded to bf16 for the tensor cores
-//   3. y[h][c] += sum_r W_down[h][n_r] hc   tensor cores, 64 h per warp step (tile_down)
+//   3. y[h][c] = sum_r W_down[h][n_r] hc    tensor cores, 64 h per warp step
 //   4. out_acc[token][h] += w_c * y         fp32 vector reductions in L2
+// bf16: one persistent CTA per SM; a producer warp gathers the 16 rows' up pieces, then their
+// down pieces, through a ring of shared-memory stages (bulk asynchronous copies, mbarriers);
+// eight consumer warps compute.  fp32: a plain CUDA-core variant with register loads.
 #include "kernels.h"
 #include "tile.cuh"
+#include "tma.cuh"
 
 namespace moe {
 namespace {
 
 constexpr int kMaxSlots = kMaxRouted + kMaxShared;
+constexpr int kRingThreads = kThreads + 64;  // 8 consumer warps, copier, meta
+constexpr int kCopier = kWarps, kMetaWarp = kWarps + 1;
 
-template <typename T>
-__global__ void __launch_bounds__(kThreads) updown_kernel(FwdParams p) {
-  __shared__ float red[kWarps][32][4];
-  __shared__ Slot s_slot[kMaxSlots];
-  __shared__ int s_item0[kMaxSlots + 1];
+// Items per slot = ceil(union rows / 16) * token tiles; exclusive prefix into s_item0[0..n],
+// with s_item0[n_slots] = total.  Whole block.
+__device__ int updown_items(const FwdParams& p, int n_slots, int* s_item0, int* scratch) {
+  const int per = (n_slots + blockDim.x - 1) / blockDim.x;
+  const int b0 = min(n_slots, (int)threadIdx.x * per), b1 = min(n_slots, b0 + per);
+  int c = 0;
+  for (int j = b0; j < b1; ++j) {
+    const int rows = __ldcg(&p.ucnt[j]);
+    const int T = __ldcg(&p.slots[j].T);
+    const int v = ((rows + kTileRows - 1) / kTileRows) * ((T + kTileTok - 1) / kTileTok);
+    s_item0[j] = v;
+    c += v;
+  }
+  int total;
+  int run = block_exclusive_scan(c, scratch, &total);
+  for (int j = b0; j < b1; ++j) {
+    const int v = s_item0[j];
+    s_item0[j] = run;
+    run += v;
+  }
+  if (threadIdx.x == 0) s_item0[n_slots] = total;
+  __syncthreads();
+  return s_item0[n_slots];
+}
+
+struct UdPos {
+  int j, tt, rg, rows;
+};
+
+__device__ __forceinline__ UdPos decode_ud_item(const FwdParams& p, const int* s_item0,
+                                                int n_slots, int item) {
+  UdPos u;
+  u.j = find_slot(s_item0, n_slots, item);
+  u.rows = __ldcg(&p.ucnt[u.j]);
+  const int nrg = (u.rows + kTileRows - 1) / kTileRows;
+  const int local = item - s_item0[u.j];
+  u.tt = local / nrg;
+  u.rg = local % nrg;
+  return u;
+}
+
+__device__ __forceinline__ int union_row(const FwdParams& p, const UdPos& u, int r) {
+  const int idx = u.rg * kTileRows + r;
+  return __ldcg(&p.ulist[(size_t)u.j * p.Imax + (idx < u.rows ? idx : u.rg * kTileRows)]);
+}
+
+struct UdMeta {
+  const __nv_bfloat16* ud;  // the expert's packed [I][2][H] block
+  int rows[kTileRows];      // union neuron of each row (a repeated valid row past the end)
+  float coef[kTileRows][kTileTok];  // SiLU(g) if the row is kept by the token's pair, else 0
+  int tok[kTileTok];        // token of each tile column (-1 past the end)
+  float w[kTileTok];        // routing weight of each tile column
+  int xb, xpar, xlast, pad;
+};
+
+__global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p, Ring rc) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ int4 s_tab[kMaxSlots];  // {expert | kind << 16, T, q0, first up/down item}
+  __shared__ int s_ucnt[kMaxSlots];
   __shared__ int scratch[33];
-  __shared__ const T* s_x[kTileTok];
-  __shared__ const T* s_up[kTileRows];
-  __shared__ const T* s_dn[kTileRows];
-  __shared__ int s_n[kTileRows];
-  __shared__ int s_rvalid[kTileRows];
-  __shared__ int s_q[kTileTok];
-  __shared__ int s_tok[kTileTok];
-  __shared__ float s_w[kTileTok];
-  __shared__ float s_coef[kTileRows][kTileTok];
-  __shared__ float s_hcf[kTileRows][kTileTok];               // fp32 variant
-  __shared__ __align__(16) uint32_t s_hcw[kTileTok][kTileRows / 2];  // bf16 pairs, token-major
+  __shared__ int s_total;
+  __shared__ int s_abort;
+  __shared__ UdMeta s_meta[kMetaRing];
+  __shared__ __align__(16) uint32_t s_hcw[2][kTileTok][kTileRows / 2];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty = full + rc.ns;
+  uint64_t* mfull = empty + rc.ns;
+  uint64_t* mempty = mfull + kMetaRing;
+  uint64_t* xfull = mempty + kMetaRing;
+  uint64_t* xempty = xfull + 2;
+  float(*red)[kWarps][4][32] = reinterpret_cast<float(*)[kWarps][4][32]>(smem + kBarBytes);
+  unsigned char* xbuf = smem + kBarBytes + kRedBytes;
+  unsigned char* ring = xbuf + rc.nxb * rc.xs_bytes;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
+  trace_point(p.trace, 3, 0);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < rc.ns; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kWarps);
+    }
+    for (int i = 0; i < kMetaRing; ++i) {
+      mbar_init(&mfull[i], 1);
+      mbar_init(&mempty[i], kWarps + 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&xfull[i], 1);
+      mbar_init(&xempty[i], kWarps);
+    }
+    s_abort = 0;
+    mbar_init_fence();
+  }
+  for (int i = threadIdx.x; i < kMetaRing * (int)(sizeof(UdMeta) / 4); i += blockDim.x)
+    reinterpret_cast<int*>(s_meta)[i] = 0;
   pdl_trigger();
   pdl_wait();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
-  const int H = p.H, Imax = p.Imax, Wmax = p.Imax / 32;
+  trace_point(p.trace, 3, 1);
   const int n_slots = ld_cg(&p.meta[kMetaSlots]);
-  // items per slot = row groups of the kept-neuron union x token tiles
   {
+    // items per slot = ceil(union rows / 16) * token tiles; exclusive prefix into s_tab[].w
     const int per = (n_slots + blockDim.x - 1) / blockDim.x;
     const int b0 = min(n_slots, (int)threadIdx.x * per), b1 = min(n_slots, b0 + per);
     int c = 0;
     for (int j = b0; j < b1; ++j) {
-      const Slot s = p.slots[j];
-      s_slot[j] = s;
-      const int rows = ld_cg(&p.ucnt[j]);
-      const int v = ((rows + kTileRows - 1) / kTileRows) * ((s.T + kTileTok - 1) / kTileTok);
-      s_item0[j] = v;
+      const Slot sl = load_slot(&p.slots[j]);
+      const int rows = __ldcg(&p.ucnt[j]);
+      s_ucnt[j] = rows;
+      const int v = ((rows + kTileRows - 1) / kTileRows) * ((sl.T + kTileTok - 1) / kTileTok);
+      s_tab[j] = make_int4(sl.expert | (sl.kind << 16), sl.T, sl.q0, v);
       c += v;
     }
     int total;
     int run = block_exclusive_scan(c, scratch, &total);
     for (int j = b0; j < b1; ++j) {
-      const int v = s_item0[j];
-      s_item0[j] = run;
+      const int v = s_tab[j].w;
+      s_tab[j].w = run;
       run += v;
     }
-    if (threadIdx.x == 0) s_item0[n_slots] = total;
+    if (threadIdx.x == 0) s_total = total;
     __syncthreads();
   }
-  const int n_items = s_item0[n_slots];
-  const T* x = static_cast<const T*>(p.x);
-  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-    const int j = find_slot(s_item0, n_slots, item);
-    const Slot s = s_slot[j];
-    const int local = item - s_item0[j];
-    const int ntt = (s.T + kTileTok - 1) / kTileTok;
-    const int rg = local / ntt, tt = local % ntt;
-    const int rows = ld_cg(&p.ucnt[j]);
-    const T* ud = s.kind == 0
-                      ? static_cast<const T*>(p.updown_r) + (size_t)s.expert * p.I * 2 * H
-                      : static_cast<const T*>(p.updown_s) + (size_t)s.expert * p.Ish * 2 * H;
-    if (threadIdx.x < kTileRows) {
-      const int r = threadIdx.x;
-      const int idx = rg * kTileRows + r;
-      const bool valid = idx < rows;
-      const int n = p.ulist[(size_t)j * Imax + (valid ? idx : rg * kTileRows)];
-      s_n[r] = n;
-      s_rvalid[r] = valid;
-      s_up[r] = ud + (size_t)n * 2 * H;
-      s_dn[r] = ud + (size_t)n * 2 * H + H;
-    } else if (threadIdx.x >= 32 && threadIdx.x < 32 + kTileTok) {
-      const int c = threadIdx.x - 32;
-      const int ti = tt * kTileTok + c;
-      if (ti < s.T) {
-        const int q = s.q0 + ti;
-        const int tok = p.pair_token[q];
-        s_q[c] = q;
-        s_tok[c] = tok;
-        s_w[c] = p.pair_w[q];
-        s_x[c] = x + (size_t)tok * H;
-      } else {
-        s_q[c] = -1;
-        s_tok[c] = -1;
-        s_w[c] = 0.f;
-        s_x[c] = nullptr;
+  const int n_items = s_total;
+  const int i0 = (int)((long long)blockIdx.x * n_items / gridDim.x);
+  const int i1 = (int)((long long)(blockIdx.x + 1) * n_items / gridDim.x);
+  const int H = p.H, Imax = p.Imax, Wmax = p.Imax / 32;
+  volatile int* abort = &s_abort;
+
+  if (warp == kMetaWarp) {
+    // ---------------- meta: rows, coefficients, tokens and token tiles, ahead of everyone
+    int xuse[2] = {0, 0};
+    if (i0 < i1) {
+      int j = find_item_slot(s_tab, n_slots, i0);
+      int nrg = (s_ucnt[j] + kTileRows - 1) / kTileRows;
+      int local = i0 - s_tab[j].w;
+      int tt = local / nrg, rg = local % nrg;
+      int key = -1, xb = rc.nxb - 1;
+      for (int item = i0, mi = 0; item < i1; ++item, ++mi) {
+        const int m = mi % kMetaRing;
+        if (!mbar_wait(&mempty[m], ((mi / kMetaRing) & 1) ^ 1, abort, p.err)) break;
+        const int4 sl = s_tab[j];
+        const int kind = sl.x >> 16, ex = sl.x & 0xffff, T = sl.y, q0 = sl.z, rows = s_ucnt[j];
+        const int nt = min(kTileTok, T - tt * kTileTok);
+        const int qt = q0 + tt * kTileTok;
+        // row of this lane (lanes 0..15) and token of this lane (lanes 0..7)
+        const int ridx = rg * kTileRows + (lane & 15);
+        const int n_l = __ldcg(&p.ulist[(size_t)j * Imax + (ridx < rows ? ridx : rg * kTileRows)]);
+        const int tok_l = lane < nt ? __ldcg(&p.pair_token[qt + lane]) : -1;
+        const float w_l = lane < nt ? __ldcg(&p.pair_w[qt + lane]) : 0.f;
+        int xpar;
+        if (j * 1024 + tt != key) {
+          key = j * 1024 + tt;
+          xb = (xb + 1) % rc.nxb;
+          if (!mbar_wait(&xempty[xb], (xuse[xb] & 1) ^ 1, abort, p.err)) break;
+          xpar = xuse[xb] & 1;
+          xuse[xb]++;
+          if (lane == 0) mbar_arrive_expect_tx(&xfull[xb], kTileTok * H * 2);
+          __syncwarp();
+          if (lane < kTileTok) {
+            const void* src = tok_l >= 0 ? static_cast<const void*>(
+                                               static_cast<const __nv_bfloat16*>(p.x) +
+                                               (size_t)tok_l * H)
+                                         : p.zero_row;
+            bulk_g2s(xbuf + xb * rc.xs_bytes + lane * rc.xs_stride, src, H * 2, &xfull[xb]);
+          }
+        } else {
+          xpar = (xuse[xb] - 1) & 1;
+        }
+        // coefficients: lane l covers row l/2, columns 4*(l&1) .. +3
+        {
+          const int r = lane >> 1, c0 = (lane & 1) * 4;
+          const int n = __shfl_sync(0xffffffffu, n_l, r);
+          const bool rvalid = rg * kTileRows + r < rows;
+          uint32_t bits[4];
+          float av[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int q = qt + c0 + c;
+            const bool ok = rvalid && c0 + c < nt;
+            bits[c] = ok ? __ldcg(&p.maskbits[(size_t)q * Wmax + (n >> 5)]) : 0u;
+            av[c] = ok ? __ldcg(&p.act[(size_t)q * Imax + n]) : 0.f;
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            s_meta[m].coef[r][c0 + c] = ((bits[c] >> (n & 31)) & 1u) ? av[c] : 0.f;
+        }
+        if (lane < kTileRows) s_meta[m].rows[lane] = n_l;
+        if (lane < kTileTok) {
+          s_meta[m].tok[lane] = tok_l;
+          s_meta[m].w[lane] = w_l;
+        }
+        // the next item, to know whether this one is the last on its token tile
+        int nj = j, ntt = tt, nrg2 = rg + 1;
+        if (nrg2 >= nrg) {
+          nrg2 = 0;
+          ++ntt;
+          if (ntt * kTileTok >= T) {
+            ntt = 0;
+            ++nj;
+            while (nj < n_slots && s_ucnt[nj] == 0) ++nj;
+          }
+        }
+        const bool last = item + 1 == i1 || nj * 1024 + ntt != key;
+        if (lane == 0) {
+          s_meta[m].ud = kind == 0 ? static_cast<const __nv_bfloat16*>(p.updown_r) +
+                                         (size_t)ex * p.I * 2 * H
+                                   : static_cast<const __nv_bfloat16*>(p.updown_s) +
+                                         (size_t)ex * p.Ish * 2 * H;
+          s_meta[m].xb = xb;
+          s_meta[m].xpar = xpar;
+          s_meta[m].xlast = last;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&mfull[m]);
+        if (nj != j && nj < n_slots) nrg = (s_ucnt[nj] + kTileRows - 1) / kTileRows;
+        j = nj;
+        tt = ntt;
+        rg = nrg2;
       }
     }
-    __syncthreads();
-    if (threadIdx.x < kTileRows * kTileTok) {
-      const int r = threadIdx.x >> 3, c = threadIdx.x & 7;
-      const int q = s_q[c], n = s_n[r];
-      float coef = 0.f;
-      if (q >= 0 && s_rvalid[r] && ((p.maskbits[(size_t)q * Wmax + (n >> 5)] >> (n & 31)) & 1u))
-        coef = p.act[(size_t)q * Imax + n];
-      s_coef[r][c] = coef;
+    for (int b = 0; b < rc.nxb; ++b)
+      if (xuse[b] > 0) mbar_drain(&xfull[b], (xuse[b] - 1) & 1);
+    return;
+  }
+
+  if (warp == kCopier) {
+    // ---------------- copier: up pieces, then down pieces, of the item's 16 rows
+    const uint32_t piece = rc.kc * 2;
+    int it = 0;
+    for (int item = i0, mi = 0; item < i1 && !*abort; ++item, ++mi) {
+      const int m = mi % kMetaRing;
+      if (!mbar_wait(&mfull[m], (mi / kMetaRing) & 1, abort, p.err)) break;
+      const __nv_bfloat16* row = s_meta[m].ud + (size_t)s_meta[m].rows[lane & 15] * 2 * H;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&mempty[m]);
+      bool stop = false;
+      for (int half = 0; half < 2 && !stop; ++half) {
+        const int rs = half ? rc.rs_d : rc.rs_a;
+        for (int kc = 0; kc < rc.nk; ++kc, ++it) {
+          const int st = it % rc.ns;
+          if (!mbar_wait(&empty[st], ((it / rc.ns) & 1) ^ 1, abort, p.err)) {
+            stop = true;
+            break;
+          }
+          if (lane == 0) mbar_arrive_expect_tx(&full[st], kTileRows * piece);
+          __syncwarp();
+          if (lane < kTileRows)
+            bulk_g2s(ring + (size_t)st * rc.stage_bytes + lane * rs, row + half * H + kc * rc.kc,
+                     piece, &full[st]);
+        }
+      }
     }
+    for (int k = it - 1; k >= 0 && k >= it - rc.ns; --k) mbar_drain(&full[k % rc.ns], (k / rc.ns) & 1);
+    return;
+  }
+
+  // ---------------- consumers
+  int it = 0, ib = 0;
+  const int nblk = rc.kc / 32, nsub = rc.kc / 64;
+  for (int item = i0, mi = 0; item < i1; ++item, ++mi) {
+    const int m = mi % kMetaRing;
+    mbar_wait(&mfull[m], (mi / kMetaRing) & 1, abort, p.err);
+    const UdMeta& mt = s_meta[m];
+    const int xb = min(max(mt.xb, 0), rc.nxb - 1);  // a record is trusted only without abort
+    const int xlast = mt.xlast;
+    const int tok0 = mt.tok[2 * t], tok1 = mt.tok[2 * t + 1];
+    const float w0 = mt.w[2 * t], w1 = mt.w[2 * t + 1];
+    mbar_wait(&xfull[xb], mt.xpar, abort, p.err);
+    const unsigned char* xrow = xbuf + xb * rc.xs_bytes + g * rc.xs_stride;
     // 1. up projection
     float d[4] = {0.f, 0.f, 0.f, 0.f};
-    tile_dot<4>(s_up[g], s_up[g + 8], s_x, warp, kWarps, H / 32, d);
+    for (int kc = 0; kc < rc.nk; ++kc, ++it) {
+      const int st = it % rc.ns;
+      mbar_wait(&full[st], (it / rc.ns) & 1, abort, p.err);
+      const unsigned char* stage = ring + (size_t)st * rc.stage_bytes;
+      for (int b = warp; b < nblk; b += kWarps) {
+        const int col = (b * 32 + t * 8) * 2;
+        const uint4 a0 = lds128(stage + g * rc.rs_a + col);
+        const uint4 a1 = lds128(stage + (g + 8) * rc.rs_a + col);
+        const uint4 xv = lds128(xrow + kc * rc.kc * 2 + col);
+        mma_16816(d, a0.x, a1.x, a0.y, a1.y, xv.x, xv.y);
+        mma_16816(d, a0.z, a1.z, a0.w, a1.w, xv.z, xv.w);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+    }
+    if (lane == 0 && xlast) mbar_arrive(&xempty[xb]);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) red[ib][warp][c][lane] = d[c];
+    const int aborted = consumer_sync_or(kThreads, *abort);
+    // 2. coefficients times u, rounded to bf16, token-major (one element per thread)
+    if (threadIdx.x < 128) {
+      const int ln = threadIdx.x & 31, c = threadIdx.x >> 5;
+      float v = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) v += red[ib][w][c][ln];
+      const int r = (ln >> 2) + (c >> 1) * 8, tok = 2 * (ln & 3) + (c & 1);
+      reinterpret_cast<__nv_bfloat16*>(&s_hcw[ib][tok][0])[r] =
+          __float2bfloat16_rn(mt.coef[r][tok] * v);
+    }
+    consumer_sync(kThreads);
+    if (lane == 0) mbar_arrive(&mempty[m]);
+    // 3-4. down projection of each stage's 64-column sub-chunks, reduced into out_acc
+    const uint32_t b0 = s_hcw[ib][g][t], b1 = s_hcw[ib][g][4 + t];
+    for (int kc = 0; kc < rc.nk; ++kc, ++it) {
+      const int st = it % rc.ns;
+      mbar_wait(&full[st], (it / rc.ns) & 1, abort, p.err);
+      const unsigned char* stage = ring + (size_t)st * rc.stage_bytes;
+      for (int sc = warp; sc < nsub; sc += kWarps) {
+        const int off = (sc * 64 + 8 * g) * 2;
+        const uint4 r0 = lds128(stage + (2 * t) * rc.rs_d + off);
+        const uint4 r1 = lds128(stage + (2 * t + 1) * rc.rs_d + off);
+        const uint4 r2 = lds128(stage + (2 * t + 8) * rc.rs_d + off);
+        const uint4 r3 = lds128(stage + (2 * t + 9) * rc.rs_d + off);
+        const uint32_t w0v[4] = {r0.x, r0.y, r0.z, r0.w}, w1v[4] = {r1.x, r1.y, r1.z, r1.w};
+        const uint32_t w2v[4] = {r2.x, r2.y, r2.z, r2.w}, w3v[4] = {r3.x, r3.y, r3.z, r3.w};
+        const int hb = kc * rc.kc + sc * 64 + 8 * g;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+          mma_16816(acc, __byte_perm(w0v[i], w1v[i], 0x5410), __byte_perm(w0v[i], w1v[i], 0x7632),
+                    __byte_perm(w2v[i], w3v[i], 0x5410), __byte_perm(w2v[i], w3v[i], 0x7632), b0,
+                    b1);
+          const int h = hb + 2 * i;
+          if (!aborted && tok0 >= 0)
+            red_add_v2(p.out_acc + (size_t)tok0 * H + h, w0 * acc[0], w0 * acc[2]);
+          if (!aborted && tok1 >= 0)
+            red_add_v2(p.out_acc + (size_t)tok1 * H + h, w1 * acc[1], w1 * acc[3]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+    }
+    ib ^= 1;
+  }
+  trace_point(p.trace, 3, 7);
+}
+
+// fp32 variant: register loads, same items and fragment layout.
+__global__ void __launch_bounds__(kThreads) updown_f32_kernel(FwdParams p) {
+  __shared__ float red[kWarps][32][4];
+  __shared__ int s_item0[kMaxSlots + 1];
+  __shared__ int scratch[33];
+  __shared__ const float* s_x[kTileTok];
+  __shared__ const float* s_up[kTileRows];
+  __shared__ const float* s_dn[kTileRows];
+  __shared__ int s_tok[kTileTok];
+  __shared__ float s_w[kTileTok];
+  __shared__ float s_coef[kTileRows][kTileTok];
+  __shared__ float s_hcf[kTileRows][kTileTok];
+  pdl_trigger();
+  pdl_wait();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
+  const int H = p.H, Imax = p.Imax, Wmax = p.Imax / 32;
+  const int n_slots = ld_cg(&p.meta[kMetaSlots]);
+  const int n_items = updown_items(p, n_slots, s_item0, scratch);
+  const float* x = static_cast<const float*>(p.x);
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    const UdPos u = decode_ud_item(p, s_item0, n_slots, item);
+    const Slot s = load_slot(&p.slots[u.j]);
+    const float* ud = s.kind == 0 ? static_cast<const float*>(p.updown_r) + (size_t)s.expert * p.I * 2 * H
+                                  : static_cast<const float*>(p.updown_s) + (size_t)s.expert * p.Ish * 2 * H;
+    if (threadIdx.x < kTileRows) {
+      const int n = union_row(p, u, threadIdx.x);
+      s_up[threadIdx.x] = ud + (size_t)n * 2 * H;
+      s_dn[threadIdx.x] = ud + (size_t)n * 2 * H + H;
+    } else if (threadIdx.x >= 32 && threadIdx.x < 32 + kTileTok) {
+      const int c = threadIdx.x - 32, ti = u.tt * kTileTok + c;
+      const bool ok = ti < s.T;
+      const int tok = ok ? __ldcg(&p.pair_token[s.q0 + ti]) : -1;
+      s_tok[c] = tok;
+      s_w[c] = ok ? __ldcg(&p.pair_w[s.q0 + ti]) : 0.f;
+      s_x[c] = ok ? x + (size_t)tok * H : nullptr;
+    }
+    if (threadIdx.x >= 64 && threadIdx.x < 64 + kTileRows * kTileTok) {
+      const int r = (threadIdx.x - 64) >> 3, c = (threadIdx.x - 64) & 7;
+      const int ti = u.tt * kTileTok + c, n = union_row(p, u, r);
+      float coef = 0.f;
+      if (ti < s.T && u.rg * kTileRows + r < u.rows) {
+        const int q = s.q0 + ti;
+        if ((__ldcg(&p.maskbits[(size_t)q * Wmax + (n >> 5)]) >> (n & 31)) & 1u)
+          coef = __ldcg(&p.act[(size_t)q * Imax + n]);
+      }
+      s_coef[r][c] = coef;
+    }
+    __syncthreads();
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+    tile_dot<1>(s_up[g], s_up[g + 8], s_x, warp, kWarps, H / 32, d);
 #pragma unroll
     for (int c = 0; c < 4; ++c) red[warp][lane][c] = d[c];
     __syncthreads();
-    // 2. coefficients
     if (warp == 0) {
       reduce_fragments(red, d);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int r = g + (c >> 1) * 8, tok = 2 * t + (c & 1);
-        const float hc = s_coef[r][tok] * d[c];
-        s_hcf[r][tok] = hc;
-        reinterpret_cast<__nv_bfloat16*>(&s_hcw[tok][0])[r] = __float2bfloat16_rn(hc);
+        s_hcf[r][tok] = s_coef[r][tok] * d[c];
       }
     }
     __syncthreads();
-    // 3-4. down projection and weighted reduction into out_acc
-    const uint32_t b0 = s_hcw[g][t], b1 = s_hcw[g][4 + t];
     const int tok0 = s_tok[2 * t], tok1 = s_tok[2 * t + 1];
     const float w0 = s_w[2 * t], w1 = s_w[2 * t + 1];
     for (int ch = warp; ch < H / 64; ch += kWarps) {
@@ -139,7 +432,7 @@ __global__ void __launch_bounds__(kThreads) updown_kernel(FwdParams p) {
       float acc[4][4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-      tile_down(s_dn, h0, b0, b1, s_hcf, acc);
+      tile_down(s_dn, h0, 0u, 0u, s_hcf, acc);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int h = h0 + 8 * g + 2 * i;
@@ -153,20 +446,32 @@ __global__ void __launch_bounds__(kThreads) updown_kernel(FwdParams p) {
 
 }  // namespace
 
-cudaError_t launch_updown(const FwdParams& p, int dtype, const LaunchShape& ls, cudaStream_t st) {
+cudaError_t launch_updown(const FwdParams& p, int dtype, const LaunchShape& ls, cudaStream_t st,
+                          bool pdl) {
   if (dtype == 0)
-    return launch_pdl(updown_kernel<__nv_bfloat16>, dim3(ls.grid_updown), dim3(kThreads), 0, st,
-                      true, p);
-  return launch_pdl(updown_kernel<float>, dim3(ls.grid_updown), dim3(kThreads), 0, st, true, p);
+    return launch_pdl(updown_tma_kernel, dim3(ls.nsm), dim3(kRingThreads), ls.ring_ud.smem_bytes,
+                      st, pdl, p, ls.ring_ud);
+  return launch_pdl(updown_f32_kernel, dim3(ls.grid_updown), dim3(kThreads), 0, st, pdl, p);
 }
 
-int updown_occupancy(int dtype) {
+Ring make_ring(int H, int smem_budget, int static_smem);
+
+cudaError_t configure_updown(int dtype, int H, int smem_budget, LaunchShape* ls) {
+  if (dtype == 0) {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, updown_tma_kernel);
+    if (e != cudaSuccess) return e;
+    ls->ring_ud = make_ring(H, smem_budget, (int)fa.sharedSizeBytes + 1024);
+    if (ls->ring_ud.ns < 2) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(updown_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ls->ring_ud.smem_bytes);
+    ls->grid_updown = ls->nsm;
+    return e;
+  }
   int n = 0;
-  if (dtype == 0)
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, updown_kernel<__nv_bfloat16>, kThreads, 0);
-  else
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, updown_kernel<float>, kThreads, 0);
-  return n;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, updown_f32_kernel, kThreads, 0);
+  ls->grid_updown = ls->nsm * (n > 0 ? n : 1);
+  return e;
 }
 
 }  // namespace moe
