@@ -10,13 +10,19 @@
 //
 // bf16: one persistent CTA per SM with three roles.
 //   meta warp    walks the items ahead of the others (at most kMetaRing): resolves each item's
-//                rows and pairs into a small shared-memory ring and, when the token tile
-//                changes, bulk-copies the 8 token rows into one of two token-tile buffers;
+//                rows and tokens into a small shared-memory ring;
 //   copier warp  streams the item's 16 gate rows, kc columns at a time, into a ring of
-//                shared-memory stages (bulk asynchronous copies completed on mbarriers);
+//                shared-memory stages (one bulk asynchronous copy per row piece, completed on an
+//                mbarrier);
 //   8 consumer warps  split each stage's columns, multiply on the tensor cores against the
 //                token tile, and sum their partial 16x8 tiles at the end of the item.
-// Consumers issue no global load: every latency is taken by a warp that runs ahead.
+// Consumers issue no global load except their token fragments when the token tile changes.
+// Template <NK, BPW>: the row is NK stages of kc = H/NK columns and warp w always takes the
+// column blocks w, w+8, ... (at most BPW per stage), so its token fragments stay in registers and
+// the whole shared memory goes to the ring.  NK = 0 is the generic variant for other H: the token
+// tile is bulk-copied into (double-buffered) shared memory by the meta warp.
+// Bulk copies of a few kilobytes per row piece reach the HBM copy rate; 1 KB copies reach about
+// half of it, which is why the pieces are as wide as shared memory allows.
 // fp32: a plain CUDA-core variant (register loads, same fragment layout).
 #include "kernels.h"
 #include "tile.cuh"
@@ -34,10 +40,14 @@ struct GateMeta {
   int q0;                     // pair index of the tile's first token
   int nt;                     // valid tokens in the tile (1..8)
   int n0;                     // first neuron
-  int xb, xpar, xlast;        // token tile buffer, its fill phase, last item using it
+  int key;                    // token tile id (slot * 1024 + tile)
+  int xb, xpar, xlast;        // generic variant: token tile buffer, fill phase, last user
+  int tok[kTileTok];          // register variant: token of each tile column (-1 past the end)
 };
 
+template <int NK, int BPW>
 __global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, Ring rc) {
+  constexpr bool kReg = NK > 0;
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int4 s_tab[kMaxSlots];
   __shared__ GateMeta s_meta[kMetaRing];
@@ -67,13 +77,10 @@ __global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, 
       mbar_init(&xempty[i], kWarps);
     }
     s_abort = 0;
-    for (int i = 0; i < kMetaRing; ++i) {
-      s_meta[i].rows = static_cast<const __nv_bfloat16*>(p.gate_r);
-      s_meta[i].q0 = s_meta[i].nt = s_meta[i].n0 = 0;
-      s_meta[i].xb = s_meta[i].xpar = s_meta[i].xlast = 0;
-    }
     mbar_init_fence();
   }
+  for (int i = threadIdx.x; i < kMetaRing * (int)(sizeof(GateMeta) / 4); i += blockDim.x)
+    reinterpret_cast<int*>(s_meta)[i] = 0;  // pointers become null, tokens 0
   pdl_trigger();
   pdl_wait();
   trace_point(p.trace, 1, 1);
@@ -87,70 +94,73 @@ __global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, 
   volatile int* abort = &s_abort;
 
   if (warp == kMetaWarp) {
-    // ---------------- meta: item records and token tiles, ahead of everyone
-    if (i0 >= i1) return;
-    int j = find_item_slot(s_tab, n_slots, i0);
-    int I = (s_tab[j].x >> 16) ? p.Ish : p.I;
-    int local = i0 - s_tab[j].w;
-    int tt = local / (I / kTileRows), rg = local % (I / kTileRows);
-    int key = -1, xb = rc.nxb - 1;
+    // ---------------- meta: item records (and, generic variant, token tiles) ahead of everyone
     int xuse[2] = {0, 0};
-    for (int item = i0, mi = 0; item < i1; ++item, ++mi) {
-      const int m = mi % kMetaRing;
-      if (!mbar_wait(&mempty[m], ((mi / kMetaRing) & 1) ^ 1, abort, p.err)) break;
-      const int4 sl = s_tab[j];
-      const int kind = sl.x >> 16, ex = sl.x & 0xffff, T = sl.y, q0 = sl.z;
-      const int nt = min(kTileTok, T - tt * kTileTok);
-      int xpar;
-      if (j * 1024 + tt != key) {
-        key = j * 1024 + tt;
-        xb = (xb + 1) % rc.nxb;
-        if (!mbar_wait(&xempty[xb], (xuse[xb] & 1) ^ 1, abort, p.err)) break;
-        xpar = xuse[xb] & 1;
-        xuse[xb]++;
-        if (lane == 0) mbar_arrive_expect_tx(&xfull[xb], kTileTok * H * 2);
+    if (i0 < i1) {
+      int j = find_item_slot(s_tab, n_slots, i0);
+      int I = (s_tab[j].x >> 16) ? p.Ish : p.I;
+      int local = i0 - s_tab[j].w;
+      int tt = local / (I / kTileRows), rg = local % (I / kTileRows);
+      int key = -1, xb = rc.nxb - 1, tok_l = -1;
+      for (int item = i0, mi = 0; item < i1; ++item, ++mi) {
+        const int m = mi % kMetaRing;
+        if (!mbar_wait(&mempty[m], ((mi / kMetaRing) & 1) ^ 1, abort, p.err)) break;
+        const int4 sl = s_tab[j];
+        const int kind = sl.x >> 16, ex = sl.x & 0xffff, T = sl.y, q0 = sl.z;
+        const int nt = min(kTileTok, T - tt * kTileTok);
+        int xpar = 0;
+        if (j * 1024 + tt != key) {
+          key = j * 1024 + tt;
+          tok_l = lane < nt ? __ldcg(&p.pair_token[q0 + tt * kTileTok + lane]) : -1;
+          if constexpr (!kReg) {
+            xb = (xb + 1) % rc.nxb;
+            if (!mbar_wait(&xempty[xb], (xuse[xb] & 1) ^ 1, abort, p.err)) break;
+            xpar = xuse[xb] & 1;
+            xuse[xb]++;
+            if (lane == 0) mbar_arrive_expect_tx(&xfull[xb], kTileTok * H * 2);
+            __syncwarp();
+            if (lane < kTileTok) {
+              const void* src = tok_l >= 0 ? static_cast<const void*>(
+                                                 static_cast<const __nv_bfloat16*>(p.x) +
+                                                 (size_t)tok_l * H)
+                                           : p.zero_row;
+              bulk_g2s(xbuf + xb * rc.xs_bytes + lane * rc.xs_stride, src, H * 2, &xfull[xb]);
+            }
+          }
+        } else if constexpr (!kReg) {
+          xpar = (xuse[xb] - 1) & 1;
+        }
+        // the next item, to know whether this one is the last on its token tile
+        int nj = j, ntt = tt, nrg = rg + 1;
+        if (nrg == I / kTileRows) {
+          nrg = 0;
+          ++ntt;
+          if (ntt * kTileTok >= T) {
+            ntt = 0;
+            ++nj;
+          }
+        }
+        if (lane < kTileTok) s_meta[m].tok[lane] = tok_l;
+        if (lane == 0) {
+          const __nv_bfloat16* base =
+              kind == 0 ? static_cast<const __nv_bfloat16*>(p.gate_r) + (size_t)ex * p.I * H
+                        : static_cast<const __nv_bfloat16*>(p.gate_s) + (size_t)ex * p.Ish * H;
+          s_meta[m].rows = base + (size_t)rg * kTileRows * H;
+          s_meta[m].q0 = q0 + tt * kTileTok;
+          s_meta[m].nt = nt;
+          s_meta[m].n0 = rg * kTileRows;
+          s_meta[m].key = key;
+          s_meta[m].xb = xb;
+          s_meta[m].xpar = xpar;
+          s_meta[m].xlast = item + 1 == i1 || nj * 1024 + ntt != key;
+        }
         __syncwarp();
-        if (lane < kTileTok) {
-          const void* src = p.zero_row;
-          if (lane < nt)
-            src = static_cast<const __nv_bfloat16*>(p.x) +
-                  (size_t)__ldcg(&p.pair_token[q0 + tt * kTileTok + lane]) * H;
-          bulk_g2s(xbuf + xb * rc.xs_bytes + lane * rc.xs_stride, src, H * 2, &xfull[xb]);
-        }
-      } else {
-        xpar = (xuse[xb] - 1) & 1;
+        if (lane == 0) mbar_arrive(&mfull[m]);
+        if (nj != j && nj < n_slots) I = (s_tab[nj].x >> 16) ? p.Ish : p.I;
+        j = nj;
+        tt = ntt;
+        rg = nrg;
       }
-      // the next item, to know whether this one is the last on its token tile
-      int nj = j, ntt = tt, nrg = rg + 1;
-      if (nrg == I / kTileRows) {
-        nrg = 0;
-        ++ntt;
-        if (ntt * kTileTok >= T) {
-          ntt = 0;
-          ++nj;
-        }
-      }
-      const bool last = item + 1 == i1 || nj * 1024 + ntt != key;
-      if (lane == 0) {
-        const __nv_bfloat16* base =
-            kind == 0 ? static_cast<const __nv_bfloat16*>(p.gate_r) + (size_t)ex * p.I * H
-                      : static_cast<const __nv_bfloat16*>(p.gate_s) + (size_t)ex * p.Ish * H;
-        GateMeta gm;
-        gm.rows = base + (size_t)rg * kTileRows * H;
-        gm.q0 = q0 + tt * kTileTok;
-        gm.nt = nt;
-        gm.n0 = rg * kTileRows;
-        gm.xb = xb;
-        gm.xpar = xpar;
-        gm.xlast = last;
-        s_meta[m] = gm;
-        mbar_arrive(&mfull[m]);
-      }
-      __syncwarp();
-      if (nj != j && nj < n_slots) I = (s_tab[nj].x >> 16) ? p.Ish : p.I;
-      j = nj;
-      tt = ntt;
-      rg = nrg;
     }
     // no token-tile copy may still be landing in shared memory when the CTA exits
     for (int b = 0; b < rc.nxb; ++b)
@@ -183,35 +193,78 @@ __global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, 
   }
 
   // ---------------- consumers
-  int it = 0, ib = 0;
+  constexpr int kXR = kReg ? NK : 1, kXB = kReg ? BPW : 1;
+  uint4 xr[kXR][kXB];
+  int it = 0, ib = 0, cur = -1;
   bool nan_seen = false;
   const int nblk = rc.kc / 32;
+  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(p.x);
   for (int item = i0, mi = 0; item < i1; ++item, ++mi) {
     const int m = mi % kMetaRing;
     mbar_wait(&mfull[m], (mi / kMetaRing) & 1, abort, p.err);
-    const GateMeta gm = s_meta[m];
-    const int xb = min(max(gm.xb, 0), rc.nxb - 1);  // a record is trusted only without abort
-    mbar_wait(&xfull[xb], gm.xpar, abort, p.err);
+    const int q0 = s_meta[m].q0, nt = s_meta[m].nt, n0 = s_meta[m].n0, key = s_meta[m].key;
+    const int xb = min(max(s_meta[m].xb, 0), max(rc.nxb - 1, 0));  // trusted only w/o abort
+    const int xlast = s_meta[m].xlast;
     const unsigned char* xrow = xbuf + xb * rc.xs_bytes + g * rc.xs_stride;
-    float d[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int kc = 0; kc < rc.nk; ++kc, ++it) {
-      const int st = it % rc.ns;
-      mbar_wait(&full[st], (it / rc.ns) & 1, abort, p.err);
-      const unsigned char* stage = ring + (size_t)st * rc.stage_bytes;
-      for (int b = warp; b < nblk; b += kWarps) {
-        const int col = (b * 32 + t * 8) * 2;
-        const uint4 a0 = lds128(stage + g * rc.rs_a + col);
-        const uint4 a1 = lds128(stage + (g + 8) * rc.rs_a + col);
-        const uint4 xv = lds128(xrow + kc * rc.kc * 2 + col);
-        mma_16816(d, a0.x, a1.x, a0.y, a1.y, xv.x, xv.y);
-        mma_16816(d, a0.z, a1.z, a0.w, a1.w, xv.z, xv.w);
+    if constexpr (kReg) {
+      if (key != cur) {  // this warp's token fragments for the new tile (one round trip)
+        cur = key;
+        const int tok = s_meta[m].tok[g];
+#pragma unroll
+        for (int kc = 0; kc < kXR; ++kc)
+#pragma unroll
+          for (int i = 0; i < kXB; ++i) {
+            const int b = warp + kWarps * i;
+            xr[kc][i] = (b < nblk && tok >= 0)
+                            ? ld_nc(x + (size_t)tok * H + kc * rc.kc + b * 32 + t * 8)
+                            : make_uint4(0, 0, 0, 0);
+          }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);
+    } else {
+      mbar_wait(&xfull[xb], s_meta[m].xpar, abort, p.err);
+    }
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+    if constexpr (kReg) {
+#pragma unroll
+      for (int kc = 0; kc < kXR; ++kc, ++it) {
+        const int st = it % rc.ns;
+        mbar_wait(&full[st], (it / rc.ns) & 1, abort, p.err);
+        const unsigned char* stage = ring + (size_t)st * rc.stage_bytes;
+#pragma unroll
+        for (int i = 0; i < kXB; ++i) {
+          const int b = warp + kWarps * i;
+          if (b < nblk) {
+            const int col = (b * 32 + t * 8) * 2;
+            const uint4 a0 = lds128(stage + g * rc.rs_a + col);
+            const uint4 a1 = lds128(stage + (g + 8) * rc.rs_a + col);
+            const uint4 xv = xr[kc][i];
+            mma_16816(d, a0.x, a1.x, a0.y, a1.y, xv.x, xv.y);
+            mma_16816(d, a0.z, a1.z, a0.w, a1.w, xv.z, xv.w);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
+      }
+    } else {
+      for (int kc = 0; kc < rc.nk; ++kc, ++it) {
+        const int st = it % rc.ns;
+        mbar_wait(&full[st], (it / rc.ns) & 1, abort, p.err);
+        const unsigned char* stage = ring + (size_t)st * rc.stage_bytes;
+        for (int b = warp; b < nblk; b += kWarps) {
+          const int col = (b * 32 + t * 8) * 2;
+          const uint4 a0 = lds128(stage + g * rc.rs_a + col);
+          const uint4 a1 = lds128(stage + (g + 8) * rc.rs_a + col);
+          const uint4 xv = lds128(xrow + kc * rc.kc * 2 + col);
+          mma_16816(d, a0.x, a1.x, a0.y, a1.y, xv.x, xv.y);
+          mma_16816(d, a0.z, a1.z, a0.w, a1.w, xv.z, xv.w);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
+      }
     }
     if (lane == 0) {
       mbar_arrive(&mempty[m]);
-      if (gm.xlast) mbar_arrive(&xempty[xb]);
+      if (!kReg && xlast) mbar_arrive(&xempty[xb]);
     }
 #pragma unroll
     for (int c = 0; c < 4; ++c) red[ib][warp][c][lane] = d[c];
@@ -223,10 +276,10 @@ __global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, 
 #pragma unroll
       for (int w = 0; w < kWarps; ++w) v += red[ib][w][c][ln];
       const int ti = 2 * (ln & 3) + (c & 1);
-      if (ti < gm.nt) {
+      if (ti < nt) {
         const float a = silu(v);
         nan_seen |= isnan(a);
-        p.act[(size_t)(gm.q0 + ti) * p.Imax + gm.n0 + (ln >> 2) + (c >> 1) * 8] = a;
+        p.act[(size_t)(q0 + ti) * p.Imax + n0 + (ln >> 2) + (c >> 1) * 8] = a;
       }
     }
     ib ^= 1;
@@ -287,17 +340,43 @@ __global__ void __launch_bounds__(kThreads) gate_f32_kernel(FwdParams p) {
   if (nan_seen) set_error(p.err, kErrNanAct);
 }
 
+template <int NK, int BPW>
+cudaError_t set_gate_smem(const Ring& r) {
+  return cudaFuncSetAttribute(gate_tma_kernel<NK, BPW>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, r.smem_bytes);
+}
+
+template <int NK, int BPW>
+int gate_static_smem() {
+  cudaFuncAttributes fa;
+  return cudaFuncGetAttributes(&fa, gate_tma_kernel<NK, BPW>) == cudaSuccess
+             ? (int)fa.sharedSizeBytes
+             : 16384;
+}
+
 }  // namespace
 
-// Copy-ring shape for hidden size H: the widest row pieces (kc a multiple of 64 dividing H) that
-// still leave two stages, two token tiles when they fit.  Bulk copies of a few kilobytes reach
-// the HBM copy rate, copies of 1 KB reach about half of it.
-Ring make_ring(int H, int smem_budget, int static_smem) {
+// Register-fragment variants, by hidden size: {H, NK, BPW}.  H = NK stages of kc columns, and
+// each of the 8 warps takes at most BPW 32-column blocks of a stage.
+extern const int kRegVariants[4][3];
+const int kRegVariants[4][3] = {{512, 1, 2}, {2048, 1, 8}, {2880, 3, 4}, {5120, 4, 5}};
+
+int ring_variant(int H) {
+  for (int v = 0; v < 4; ++v)
+    if (kRegVariants[v][0] == H) return v + 1;
+  return 0;
+}
+
+// Copy-ring shape.  Register variant (nk_fixed > 0): the whole budget goes to stages of kc =
+// H/nk_fixed.  Generic variant (nk_fixed = 0): the widest row pieces (kc a multiple of 64
+// dividing H) that still leave two stages next to two token tiles (or one).
+Ring make_ring(int H, int nk_fixed, int smem_budget, int static_smem) {
   const int avail = smem_budget - static_smem - kBarBytes - kRedBytes;
-  Ring best{};
-  best.ns = 0;
-  for (int nk = 1; nk <= H / 64; ++nk) {
-    if (H % nk || (H / nk) % 64) continue;
+  for (int nk = nk_fixed ? nk_fixed : 1; nk <= H / 64; ++nk) {
+    if (H % nk || (H / nk) % 64) {
+      if (nk_fixed) break;
+      continue;
+    }
     Ring r;
     r.nk = nk;
     r.kc = H / nk;
@@ -306,7 +385,7 @@ Ring make_ring(int H, int smem_budget, int static_smem) {
     r.stage_bytes = kTileRows * r.rs_a;
     r.xs_stride = H * 2 + 64;
     r.xs_bytes = kTileTok * r.xs_stride;
-    for (int nxb = 2; nxb >= 1; --nxb) {
+    for (int nxb = nk_fixed ? 0 : 2; nxb >= (nk_fixed ? 0 : 1); --nxb) {
       int ns = (avail - nxb * r.xs_bytes) / r.stage_bytes;
       if (ns > 16) ns = 16;
       if (ns >= 2) {
@@ -316,34 +395,55 @@ Ring make_ring(int H, int smem_budget, int static_smem) {
         return r;
       }
     }
+    if (nk_fixed) break;
   }
-  return best;  // ns == 0: no ring fits
+  Ring none{};
+  none.ns = 0;
+  return none;
 }
 
 cudaError_t launch_gate(const FwdParams& p, int dtype, const LaunchShape& ls, cudaStream_t st,
                         bool pdl) {
-  if (dtype == 0)
-    return launch_pdl(gate_tma_kernel, dim3(ls.nsm), dim3(kRingThreads), ls.ring_gate.smem_bytes,
-                      st, pdl, p, ls.ring_gate);
-  return launch_pdl(gate_f32_kernel, dim3(ls.grid_gate), dim3(kThreads), 0, st, pdl, p);
+  if (dtype != 0)
+    return launch_pdl(gate_f32_kernel, dim3(ls.grid_gate), dim3(kThreads), 0, st, pdl, p);
+  const Ring& r = ls.ring_gate;
+  const dim3 grid(ls.nsm), block(kRingThreads);
+  switch (ls.variant) {
+    case 1: return launch_pdl(gate_tma_kernel<1, 2>, grid, block, r.smem_bytes, st, pdl, p, r);
+    case 2: return launch_pdl(gate_tma_kernel<1, 8>, grid, block, r.smem_bytes, st, pdl, p, r);
+    case 3: return launch_pdl(gate_tma_kernel<3, 4>, grid, block, r.smem_bytes, st, pdl, p, r);
+    case 4: return launch_pdl(gate_tma_kernel<4, 5>, grid, block, r.smem_bytes, st, pdl, p, r);
+    default: return launch_pdl(gate_tma_kernel<0, 0>, grid, block, r.smem_bytes, st, pdl, p, r);
+  }
 }
 
 cudaError_t configure_gate(int dtype, int H, int smem_budget, LaunchShape* ls) {
-  if (dtype == 0) {
-    cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, gate_tma_kernel);
-    if (e != cudaSuccess) return e;
-    ls->ring_gate = make_ring(H, smem_budget, (int)fa.sharedSizeBytes + 1024);
-    if (ls->ring_gate.ns < 2) return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(gate_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             ls->ring_gate.smem_bytes);
-    ls->grid_gate = ls->nsm;
+  if (dtype != 0) {
+    int n = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gate_f32_kernel, kThreads, 0);
+    ls->grid_gate = ls->nsm * (n > 0 ? n : 1);
     return e;
   }
-  int n = 0;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gate_f32_kernel, kThreads, 0);
-  ls->grid_gate = ls->nsm * (n > 0 ? n : 1);
-  return e;
+  ls->variant = ring_variant(H);
+  const int nk = ls->variant ? kRegVariants[ls->variant - 1][1] : 0;
+  int stat = 0;
+  switch (ls->variant) {
+    case 1: stat = gate_static_smem<1, 2>(); break;
+    case 2: stat = gate_static_smem<1, 8>(); break;
+    case 3: stat = gate_static_smem<3, 4>(); break;
+    case 4: stat = gate_static_smem<4, 5>(); break;
+    default: stat = gate_static_smem<0, 0>(); break;
+  }
+  ls->ring_gate = make_ring(H, nk, smem_budget, stat + 1024);
+  if (ls->ring_gate.ns < 2) return cudaErrorInvalidConfiguration;
+  ls->grid_gate = ls->nsm;
+  switch (ls->variant) {
+    case 1: return set_gate_smem<1, 2>(ls->ring_gate);
+    case 2: return set_gate_smem<1, 8>(ls->ring_gate);
+    case 3: return set_gate_smem<3, 4>(ls->ring_gate);
+    case 4: return set_gate_smem<4, 5>(ls->ring_gate);
+    default: return set_gate_smem<0, 0>(ls->ring_gate);
+  }
 }
 
 }  // namespace moe

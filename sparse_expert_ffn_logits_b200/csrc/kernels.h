@@ -15,6 +15,7 @@ struct LaunchShape {
   int grid_select;    // cap of the selection grid
   Ring ring_gate;     // copy ring of the bf16 gate kernel
   Ring ring_ud;       // copy ring of the bf16 up/down kernel
+  int variant;        // register-fragment ring variant (0: generic token tiles in smem)
 };
 
 // dtype: 0 bf16, 1 fp32.  Each launcher returns the launch's cudaError_t.

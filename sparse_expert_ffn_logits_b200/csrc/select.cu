@@ -3,16 +3,16 @@
 // Inside a pair the lowest-scoring neuron activations are dropped ("Uncovering Intra-expert
 // Activation Sparsity ...", technical summary, Methodology: activation masking).  The score of
 // neuron n is |SiLU(g_n)|, an fp32 value whose bit pattern (sign cleared) orders like the value.
-//   top-K mode: an MSB-first radix select (four 8-bit digits) finds the K-th largest key tau
+//   top-K mode: an MSB-first radix select (eight 4-bit digits) finds the K-th largest key tau
 //     and how many keys equal to tau are kept; the kept set is every key > tau plus the
 //     lowest-indexed keys == tau.  No sort.
 //   threshold mode: one pass, keep key > t (the page's single-pass threshold mask).
-// One CTA per pair: its keys sit in shared memory; each warp histograms its share of them into
-// its own 256 bins (lanes holding the same digit are merged by a match-any vote, one plain add
-// per distinct digit), and a block scan over the summed bins finds the digit.  The kept set is
-// written as an ascending index list + count (for export), as a bitmask row, and OR-ed into the
-// expert's union bitmask.  The last pair of an expert to finish (atomic ticket, no waiting)
-// compacts the union into an ascending row list for the up/down kernel and clears the bitmask.
+// One CTA per pair: its keys sit in shared memory; each radix pass counts digits in registers
+// (packed 16-bit bins) and merges them with warp reductions, with no atomics.  The kept set is
+// written as an ascending index list + count (for export), as a bitmask row, and
+// OR-ed into the expert's union bitmask.  The last pair of an expert to finish (atomic ticket,
+// no waiting) compacts the union into an ascending row list for the up/down kernel and clears
+// the bitmask.
 #include "kernels.h"
 
 namespace moe {
@@ -23,7 +23,7 @@ constexpr int kSelWarps = kSelThreads / 32;
 
 __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
   extern __shared__ uint32_t sm[];
-  __shared__ int hist[kSelWarps][256];
+  __shared__ int hist[2048];
   __shared__ int scratch[33];
   __shared__ int wtot[kSelWarps];
   __shared__ int s_digit, s_above, s_last;
@@ -68,6 +68,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
       }
     }
     __syncthreads();
+    if (q == (int)blockIdx.x) trace_point(p.trace, 2, 2);
     const int mode = p.sel_mode[kind];
     const int K = min(p.sel_K[kind], I);
     const float thr = p.sel_t[kind];
@@ -75,40 +76,54 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
     uint32_t tau = 0;
     int need = 0;
     if (radix) {
+      // eight 4-bit digits, most significant first.  Each thread counts its keys per digit in
+      // packed 16-bit fields (bins 2i, 2i+1 in c[i]), a warp sum merges them, and warp 0 reads
+      // the eight warps' sums to pick the digit: no atomics, two barriers per digit.
       uint32_t prefix = 0, pmask = 0;
       int krem = K;
-      for (int shift = 24; shift >= 0; shift -= 8) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) hist[warp][lane * 8 + i] = 0;
-        __syncwarp();
-        for (int n = warp * 32 + lane; n < I; n += kSelThreads) {
+#pragma unroll 1
+      for (int shift = 28; shift >= 0; shift -= 4) {
+        uint32_t c[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        for (int n = threadIdx.x; n < I; n += blockDim.x) {
           const uint32_t u = key[n];
-          const bool match = (u & pmask) == prefix;
-          const uint32_t dg = match ? (u >> shift) & 255u : 256u + lane;
-          const unsigned same = __match_any_sync(0xffffffffu, dg);
-          if (match && lane == __ffs(same) - 1) hist[warp][dg] += __popc(same);
-          __syncwarp();
+          if ((u & pmask) == prefix) {
+            const uint32_t d = (u >> shift) & 15u;
+            const uint32_t inc = 1u << ((d & 1u) * 16);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) c[i] += (d >> 1) == (uint32_t)i ? inc : 0u;
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) c[i] = __reduce_add_sync(0xffffffffu, c[i]);
+        if (lane == 0) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) hist[warp * 8 + i] = (int)c[i];
         }
         __syncthreads();
-        // thread b holds digit 255 - b (descending order), summed over the warps
-        const int dig = 255 - (int)threadIdx.x;
-        int c = 0;
-#pragma unroll
-        for (int w = 0; w < kSelWarps; ++w) c += hist[w][dig];
-        int total;
-        const int above = block_exclusive_scan(c, scratch, &total);
-        if (above < krem && above + c >= krem) {
-          s_digit = dig;
+        if (threadIdx.x == 0) {
+          int above = 0, digit = 0;
+          for (int d = 15; d >= 0; --d) {
+            int cnt = 0;
+            for (int w = 0; w < kSelWarps; ++w)
+              cnt += (int)(((uint32_t)hist[w * 8 + (d >> 1)] >> ((d & 1) * 16)) & 0xFFFFu);
+            if (above + cnt >= krem) {
+              digit = d;
+              break;
+            }
+            above += cnt;
+          }
+          s_digit = digit;
           s_above = above;
         }
         __syncthreads();
         krem -= s_above;
         prefix |= (uint32_t)s_digit << shift;
-        pmask |= 255u << shift;
+        pmask |= 15u << shift;
       }
       tau = prefix;
       need = krem;
     }
+    if (q == (int)blockIdx.x) trace_point(p.trace, 2, 3);
     // warp-contiguous segments of the neuron range, walked 32 at a time (ordered ballots)
     const int seg = ((I + 32 * kSelWarps - 1) / (32 * kSelWarps)) * 32;
     const int sb = warp * seg, se = min(I, sb + seg);
@@ -170,13 +185,16 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
       }
     }
     if (threadIdx.x == 0) p.cnt[q] = total;
+    if (q == (int)blockIdx.x) trace_point(p.trace, 2, 4);
     __threadfence();
     __syncthreads();
+    if (q == (int)blockIdx.x) trace_point(p.trace, 2, 5);
     if (threadIdx.x == 0) {
       const unsigned ticket = atomicAdd(&p.slot_ticket[j], 1u);
       s_last = ticket == (unsigned)s.T - 1u;
     }
     __syncthreads();
+    if (q == (int)blockIdx.x) trace_point(p.trace, 2, 6);
     if (s_last) {
       // last pair of this expert: compact the union bitmask into a row list, clear it
       __threadfence();

@@ -24,8 +24,11 @@ namespace moe {
 namespace {
 
 constexpr int kMaxSlots = kMaxRouted + kMaxShared;
-constexpr int kRingThreads = kThreads + 64;  // 8 consumer warps, copier, meta
-constexpr int kCopier = kWarps, kMetaWarp = kWarps + 1;
+// 8 consumer warps, the copier, the lead meta warp (token tiles) and kCoefWarps coefficient
+// warps that fill alternate item records in parallel (each record costs two dependent L2 reads)
+constexpr int kCoefWarps = 2;
+constexpr int kRingThreads = kThreads + 64 + 32 * kCoefWarps;
+constexpr int kCopier = kWarps, kMetaWarp = kWarps + 1, kCoefWarp0 = kWarps + 2;
 
 // Items per slot = ceil(union rows / 16) * token tiles; exclusive prefix into s_item0[0..n],
 // with s_item0[n_slots] = total.  Whole block.
@@ -79,10 +82,13 @@ struct UdMeta {
   float coef[kTileRows][kTileTok];  // SiLU(g) if the row is kept by the token's pair, else 0
   int tok[kTileTok];        // token of each tile column (-1 past the end)
   float w[kTileTok];        // routing weight of each tile column
-  int xb, xpar, xlast, pad;
+  int key;                  // token tile id (slot * 1024 + tile)
+  int xb, xpar, xlast;      // generic variant: token tile buffer, fill phase, last user
 };
 
+template <int NK, int BPW>
 __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p, Ring rc) {
+  constexpr bool kReg = NK > 0;
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int4 s_tab[kMaxSlots];  // {expert | kind << 16, T, q0, first up/down item}
   __shared__ int s_ucnt[kMaxSlots];
@@ -108,7 +114,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
       mbar_init(&empty[i], kWarps);
     }
     for (int i = 0; i < kMetaRing; ++i) {
-      mbar_init(&mfull[i], 1);
+      mbar_init(&mfull[i], 2);  // lead meta warp + the coefficient warp of that record
       mbar_init(&mempty[i], kWarps + 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -153,8 +159,12 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
   const int H = p.H, Imax = p.Imax, Wmax = p.Imax / 32;
   volatile int* abort = &s_abort;
 
-  if (warp == kMetaWarp) {
-    // ---------------- meta: rows, coefficients, tokens and token tiles, ahead of everyone
+  if (warp >= kMetaWarp) {
+    // ---------------- meta warps: walk the items ahead of the copier and the consumers.
+    // The lead warp owns the token tiles (and the record fields ud, xb, xpar, xlast); coefficient
+    // warp c owns rows, coef, tok and w of the records mi with mi % kCoefWarps == c.
+    const bool lead = warp == kMetaWarp;
+    const int cw = warp - kCoefWarp0;
     int xuse[2] = {0, 0};
     if (i0 < i1) {
       int j = find_item_slot(s_tab, n_slots, i0);
@@ -164,37 +174,68 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
       int key = -1, xb = rc.nxb - 1;
       for (int item = i0, mi = 0; item < i1; ++item, ++mi) {
         const int m = mi % kMetaRing;
-        if (!mbar_wait(&mempty[m], ((mi / kMetaRing) & 1) ^ 1, abort, p.err)) break;
         const int4 sl = s_tab[j];
         const int kind = sl.x >> 16, ex = sl.x & 0xffff, T = sl.y, q0 = sl.z, rows = s_ucnt[j];
         const int nt = min(kTileTok, T - tt * kTileTok);
         const int qt = q0 + tt * kTileTok;
-        // row of this lane (lanes 0..15) and token of this lane (lanes 0..7)
-        const int ridx = rg * kTileRows + (lane & 15);
-        const int n_l = __ldcg(&p.ulist[(size_t)j * Imax + (ridx < rows ? ridx : rg * kTileRows)]);
-        const int tok_l = lane < nt ? __ldcg(&p.pair_token[qt + lane]) : -1;
-        const float w_l = lane < nt ? __ldcg(&p.pair_w[qt + lane]) : 0.f;
-        int xpar;
-        if (j * 1024 + tt != key) {
-          key = j * 1024 + tt;
-          xb = (xb + 1) % rc.nxb;
-          if (!mbar_wait(&xempty[xb], (xuse[xb] & 1) ^ 1, abort, p.err)) break;
-          xpar = xuse[xb] & 1;
-          xuse[xb]++;
-          if (lane == 0) mbar_arrive_expect_tx(&xfull[xb], kTileTok * H * 2);
-          __syncwarp();
-          if (lane < kTileTok) {
-            const void* src = tok_l >= 0 ? static_cast<const void*>(
-                                               static_cast<const __nv_bfloat16*>(p.x) +
-                                               (size_t)tok_l * H)
-                                         : p.zero_row;
-            bulk_g2s(xbuf + xb * rc.xs_bytes + lane * rc.xs_stride, src, H * 2, &xfull[xb]);
+        // the next item, to know whether this one is the last on its token tile
+        int nj = j, ntt = tt, nrg2 = rg + 1;
+        if (nrg2 >= nrg) {
+          nrg2 = 0;
+          ++ntt;
+          if (ntt * kTileTok >= T) {
+            ntt = 0;
+            ++nj;
+            while (nj < n_slots && s_ucnt[nj] == 0) ++nj;
           }
-        } else {
-          xpar = (xuse[xb] - 1) & 1;
         }
-        // coefficients: lane l covers row l/2, columns 4*(l&1) .. +3
-        {
+        const bool mine = lead || mi % kCoefWarps == cw;
+        if (mine) {
+          if (!mbar_wait(&mempty[m], ((mi / kMetaRing) & 1) ^ 1, abort, p.err)) break;
+        }
+        if (lead) {
+          int xpar = 0;
+          if (j * 1024 + tt != key) {
+            key = j * 1024 + tt;
+            if constexpr (!kReg) {
+              xb = (xb + 1) % rc.nxb;
+              if (!mbar_wait(&xempty[xb], (xuse[xb] & 1) ^ 1, abort, p.err)) break;
+              xpar = xuse[xb] & 1;
+              xuse[xb]++;
+              const int tok_l = lane < nt ? __ldcg(&p.pair_token[qt + lane]) : -1;
+              if (lane == 0) mbar_arrive_expect_tx(&xfull[xb], kTileTok * H * 2);
+              __syncwarp();
+              if (lane < kTileTok) {
+                const void* src = tok_l >= 0 ? static_cast<const void*>(
+                                                   static_cast<const __nv_bfloat16*>(p.x) +
+                                                   (size_t)tok_l * H)
+                                             : p.zero_row;
+                bulk_g2s(xbuf + xb * rc.xs_bytes + lane * rc.xs_stride, src, H * 2, &xfull[xb]);
+              }
+            }
+          } else if constexpr (!kReg) {
+            xpar = (xuse[xb] - 1) & 1;
+          }
+          if (lane == 0) {
+            s_meta[m].ud = kind == 0 ? static_cast<const __nv_bfloat16*>(p.updown_r) +
+                                           (size_t)ex * p.I * 2 * H
+                                     : static_cast<const __nv_bfloat16*>(p.updown_s) +
+                                           (size_t)ex * p.Ish * 2 * H;
+            s_meta[m].key = key;
+            s_meta[m].xb = xb;
+            s_meta[m].xpar = xpar;
+            s_meta[m].xlast = item + 1 == i1 || nj * 1024 + ntt != key;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&mfull[m]);
+        } else if (mine) {
+          // row of this lane (lanes 0..15) and token of this lane (lanes 0..7)
+          const int ridx = rg * kTileRows + (lane & 15);
+          const int n_l =
+              __ldcg(&p.ulist[(size_t)j * Imax + (ridx < rows ? ridx : rg * kTileRows)]);
+          const int tok_l = lane < nt ? __ldcg(&p.pair_token[qt + lane]) : -1;
+          const float w_l = lane < nt ? __ldcg(&p.pair_w[qt + lane]) : 0.f;
+          // coefficients: lane l covers row l/2, columns 4*(l&1) .. +3
           const int r = lane >> 1, c0 = (lane & 1) * 4;
           const int n = __shfl_sync(0xffffffffu, n_l, r);
           const bool rvalid = rg * kTileRows + r < rows;
@@ -210,43 +251,23 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
 #pragma unroll
           for (int c = 0; c < 4; ++c)
             s_meta[m].coef[r][c0 + c] = ((bits[c] >> (n & 31)) & 1u) ? av[c] : 0.f;
-        }
-        if (lane < kTileRows) s_meta[m].rows[lane] = n_l;
-        if (lane < kTileTok) {
-          s_meta[m].tok[lane] = tok_l;
-          s_meta[m].w[lane] = w_l;
-        }
-        // the next item, to know whether this one is the last on its token tile
-        int nj = j, ntt = tt, nrg2 = rg + 1;
-        if (nrg2 >= nrg) {
-          nrg2 = 0;
-          ++ntt;
-          if (ntt * kTileTok >= T) {
-            ntt = 0;
-            ++nj;
-            while (nj < n_slots && s_ucnt[nj] == 0) ++nj;
+          if (lane < kTileRows) s_meta[m].rows[lane] = n_l;
+          if (lane < kTileTok) {
+            s_meta[m].tok[lane] = tok_l;
+            s_meta[m].w[lane] = w_l;
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&mfull[m]);
         }
-        const bool last = item + 1 == i1 || nj * 1024 + ntt != key;
-        if (lane == 0) {
-          s_meta[m].ud = kind == 0 ? static_cast<const __nv_bfloat16*>(p.updown_r) +
-                                         (size_t)ex * p.I * 2 * H
-                                   : static_cast<const __nv_bfloat16*>(p.updown_s) +
-                                         (size_t)ex * p.Ish * 2 * H;
-          s_meta[m].xb = xb;
-          s_meta[m].xpar = xpar;
-          s_meta[m].xlast = last;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&mfull[m]);
         if (nj != j && nj < n_slots) nrg = (s_ucnt[nj] + kTileRows - 1) / kTileRows;
         j = nj;
         tt = ntt;
         rg = nrg2;
       }
     }
-    for (int b = 0; b < rc.nxb; ++b)
-      if (xuse[b] > 0) mbar_drain(&xfull[b], (xuse[b] - 1) & 1);
+    if (lead)
+      for (int b = 0; b < rc.nxb; ++b)
+        if (xuse[b] > 0) mbar_drain(&xfull[b], (xuse[b] - 1) & 1);
     return;
   }
 
@@ -282,36 +303,78 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
   }
 
   // ---------------- consumers
-  int it = 0, ib = 0;
+  constexpr int kXR = kReg ? NK : 1, kXB = kReg ? BPW : 1;
+  uint4 xr[kXR][kXB];
+  int it = 0, ib = 0, cur = -1;
   const int nblk = rc.kc / 32, nsub = rc.kc / 64;
+  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(p.x);
   for (int item = i0, mi = 0; item < i1; ++item, ++mi) {
     const int m = mi % kMetaRing;
     mbar_wait(&mfull[m], (mi / kMetaRing) & 1, abort, p.err);
     const UdMeta& mt = s_meta[m];
-    const int xb = min(max(mt.xb, 0), rc.nxb - 1);  // a record is trusted only without abort
+    const int xb = min(max(mt.xb, 0), max(rc.nxb - 1, 0));  // a record is trusted only w/o abort
     const int xlast = mt.xlast;
     const int tok0 = mt.tok[2 * t], tok1 = mt.tok[2 * t + 1];
     const float w0 = mt.w[2 * t], w1 = mt.w[2 * t + 1];
-    mbar_wait(&xfull[xb], mt.xpar, abort, p.err);
     const unsigned char* xrow = xbuf + xb * rc.xs_bytes + g * rc.xs_stride;
+    if constexpr (kReg) {
+      if (mt.key != cur) {  // this warp's token fragments for the new tile (one round trip)
+        cur = mt.key;
+        const int tok = mt.tok[g];
+#pragma unroll
+        for (int kc = 0; kc < kXR; ++kc)
+#pragma unroll
+          for (int i = 0; i < kXB; ++i) {
+            const int b = warp + kWarps * i;
+            xr[kc][i] = (b < nblk && tok >= 0)
+                            ? ld_nc(x + (size_t)tok * H + kc * rc.kc + b * 32 + t * 8)
+                            : make_uint4(0, 0, 0, 0);
+          }
+      }
+    } else {
+      mbar_wait(&xfull[xb], mt.xpar, abort, p.err);
+    }
     // 1. up projection
     float d[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int kc = 0; kc < rc.nk; ++kc, ++it) {
-      const int st = it % rc.ns;
-      mbar_wait(&full[st], (it / rc.ns) & 1, abort, p.err);
-      const unsigned char* stage = ring + (size_t)st * rc.stage_bytes;
-      for (int b = warp; b < nblk; b += kWarps) {
-        const int col = (b * 32 + t * 8) * 2;
-        const uint4 a0 = lds128(stage + g * rc.rs_a + col);
-        const uint4 a1 = lds128(stage + (g + 8) * rc.rs_a + col);
-        const uint4 xv = lds128(xrow + kc * rc.kc * 2 + col);
-        mma_16816(d, a0.x, a1.x, a0.y, a1.y, xv.x, xv.y);
-        mma_16816(d, a0.z, a1.z, a0.w, a1.w, xv.z, xv.w);
+    if constexpr (kReg) {
+#pragma unroll
+      for (int kc = 0; kc < kXR; ++kc, ++it) {
+        const int st = it % rc.ns;
+        mbar_wait(&full[st], (it / rc.ns) & 1, abort, p.err);
+        const unsigned char* stage = ring + (size_t)st * rc.stage_bytes;
+#pragma unroll
+        for (int i = 0; i < kXB; ++i) {
+          const int b = warp + kWarps * i;
+          if (b < nblk) {
+            const int col = (b * 32 + t * 8) * 2;
+            const uint4 a0 = lds128(stage + g * rc.rs_a + col);
+            const uint4 a1 = lds128(stage + (g + 8) * rc.rs_a + col);
+            const uint4 xv = xr[kc][i];
+            mma_16816(d, a0.x, a1.x, a0.y, a1.y, xv.x, xv.y);
+            mma_16816(d, a0.z, a1.z, a0.w, a1.w, xv.z, xv.w);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);
+    } else {
+      for (int kc = 0; kc < rc.nk; ++kc, ++it) {
+        const int st = it % rc.ns;
+        mbar_wait(&full[st], (it / rc.ns) & 1, abort, p.err);
+        const unsigned char* stage = ring + (size_t)st * rc.stage_bytes;
+        for (int b = warp; b < nblk; b += kWarps) {
+          const int col = (b * 32 + t * 8) * 2;
+          const uint4 a0 = lds128(stage + g * rc.rs_a + col);
+          const uint4 a1 = lds128(stage + (g + 8) * rc.rs_a + col);
+          const uint4 xv = lds128(xrow + kc * rc.kc * 2 + col);
+          mma_16816(d, a0.x, a1.x, a0.y, a1.y, xv.x, xv.y);
+          mma_16816(d, a0.z, a1.z, a0.w, a1.w, xv.z, xv.w);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
+      }
     }
-    if (lane == 0 && xlast) mbar_arrive(&xempty[xb]);
+    if (!kReg && lane == 0 && xlast) mbar_arrive(&xempty[xb]);
 #pragma unroll
     for (int c = 0; c < 4; ++c) red[ib][warp][c][lane] = d[c];
     const int aborted = consumer_sync_or(kThreads, *abort);
@@ -446,32 +509,66 @@ __global__ void __launch_bounds__(kThreads) updown_f32_kernel(FwdParams p) {
 
 }  // namespace
 
-cudaError_t launch_updown(const FwdParams& p, int dtype, const LaunchShape& ls, cudaStream_t st,
-                          bool pdl) {
-  if (dtype == 0)
-    return launch_pdl(updown_tma_kernel, dim3(ls.nsm), dim3(kRingThreads), ls.ring_ud.smem_bytes,
-                      st, pdl, p, ls.ring_ud);
-  return launch_pdl(updown_f32_kernel, dim3(ls.grid_updown), dim3(kThreads), 0, st, pdl, p);
+template <int NK, int BPW>
+cudaError_t set_ud_smem(const Ring& r) {
+  return cudaFuncSetAttribute(updown_tma_kernel<NK, BPW>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, r.smem_bytes);
 }
 
-Ring make_ring(int H, int smem_budget, int static_smem);
+template <int NK, int BPW>
+int ud_static_smem() {
+  cudaFuncAttributes fa;
+  return cudaFuncGetAttributes(&fa, updown_tma_kernel<NK, BPW>) == cudaSuccess
+             ? (int)fa.sharedSizeBytes
+             : 16384;
+}
+
+cudaError_t launch_updown(const FwdParams& p, int dtype, const LaunchShape& ls, cudaStream_t st,
+                          bool pdl) {
+  if (dtype != 0)
+    return launch_pdl(updown_f32_kernel, dim3(ls.grid_updown), dim3(kThreads), 0, st, pdl, p);
+  const Ring& r = ls.ring_ud;
+  const dim3 grid(ls.nsm), block(kRingThreads);
+  switch (ls.variant) {
+    case 1: return launch_pdl(updown_tma_kernel<1, 2>, grid, block, r.smem_bytes, st, pdl, p, r);
+    case 2: return launch_pdl(updown_tma_kernel<1, 8>, grid, block, r.smem_bytes, st, pdl, p, r);
+    case 3: return launch_pdl(updown_tma_kernel<3, 4>, grid, block, r.smem_bytes, st, pdl, p, r);
+    case 4: return launch_pdl(updown_tma_kernel<4, 5>, grid, block, r.smem_bytes, st, pdl, p, r);
+    default: return launch_pdl(updown_tma_kernel<0, 0>, grid, block, r.smem_bytes, st, pdl, p, r);
+  }
+}
+
+extern const int kRegVariants[4][3];
+Ring make_ring(int H, int nk_fixed, int smem_budget, int static_smem);
 
 cudaError_t configure_updown(int dtype, int H, int smem_budget, LaunchShape* ls) {
-  if (dtype == 0) {
-    cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, updown_tma_kernel);
-    if (e != cudaSuccess) return e;
-    ls->ring_ud = make_ring(H, smem_budget, (int)fa.sharedSizeBytes + 1024);
-    if (ls->ring_ud.ns < 2) return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(updown_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             ls->ring_ud.smem_bytes);
-    ls->grid_updown = ls->nsm;
+  if (dtype != 0) {
+    int n = 0;
+    cudaError_t e =
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, updown_f32_kernel, kThreads, 0);
+    ls->grid_updown = ls->nsm * (n > 0 ? n : 1);
     return e;
   }
-  int n = 0;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, updown_f32_kernel, kThreads, 0);
-  ls->grid_updown = ls->nsm * (n > 0 ? n : 1);
-  return e;
+  // ls->variant was chosen by configure_gate for the same H
+  const int nk = ls->variant ? kRegVariants[ls->variant - 1][1] : 0;
+  int stat = 0;
+  switch (ls->variant) {
+    case 1: stat = ud_static_smem<1, 2>(); break;
+    case 2: stat = ud_static_smem<1, 8>(); break;
+    case 3: stat = ud_static_smem<3, 4>(); break;
+    case 4: stat = ud_static_smem<4, 5>(); break;
+    default: stat = ud_static_smem<0, 0>(); break;
+  }
+  ls->ring_ud = make_ring(H, nk, smem_budget, stat + 1024);
+  if (ls->ring_ud.ns < 2) return cudaErrorInvalidConfiguration;
+  ls->grid_updown = ls->nsm;
+  switch (ls->variant) {
+    case 1: return set_ud_smem<1, 2>(ls->ring_ud);
+    case 2: return set_ud_smem<1, 8>(ls->ring_ud);
+    case 3: return set_ud_smem<3, 4>(ls->ring_ud);
+    case 4: return set_ud_smem<4, 5>(ls->ring_ud);
+    default: return set_ud_smem<0, 0>(ls->ring_ud);
+  }
 }
 
 }  // namespace moe
