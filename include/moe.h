@@ -159,13 +159,15 @@ moe_status moe_profile_stages(moe_handle* h, void* const* events, int n_events);
 
 /* Phase timestamps of the last calls made while stage timing was on (%globaltimer ns, 0 where a
  * point was not reached): host[(kernel * 1024 + cta) * 8 + point] for kernel 0..4 in launch
- * order and the first 1024 CTAs.  Synchronises the device, copies min(n, 5*1024*8) values into
+ * order and the first 1024 CTAs.  In the gate and up/down kernels point 5 holds a count (the
+ * CTA's work items), not a time.  Synchronises the device, copies min(n, 5*1024*8) values into
  * host memory, then clears the device buffer. */
 moe_status moe_read_trace(moe_handle* h, unsigned long long* host, size_t n);
 
 /* Synchronises the device, reads and clears the device error word.  Returns MOE_ERR_DEVICE
- * (code in *device_code: 1 = NaN router logit, 2 = NaN activation) if it was set, else MOE_OK
- * with *device_code = 0. */
+ * (code in *device_code: 1 = NaN router logit, 2 = NaN activation, 3 = a bounded wait inside a
+ * kernel gave up after 0.2 s; the output of that call is then invalid) if it was set, else
+ * MOE_OK with *device_code = 0. */
 moe_status moe_get_error(moe_handle* h, int* device_code);
 
 /* Frees the workspace and the handle (synchronises the device first).  NULL is a no-op. */

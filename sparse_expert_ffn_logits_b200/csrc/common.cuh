@@ -95,6 +95,7 @@ struct FwdParams {
   int* err;            // device error word
   const void* zero_row;  // H zero elements (source of the copies of absent tokens)
   unsigned long long* trace;  // per-CTA phase timestamps (nullptr: tracing off)
+  unsigned* claim;            // [2] work-item counters of the gate and up/down kernels
 };
 
 // Phase timestamps for tracing: kernel k, CTA b, point i (i < kTracePoints).
@@ -106,6 +107,14 @@ __device__ __forceinline__ void trace_point(const unsigned long long* tr_base, i
     const_cast<unsigned long long*>(tr_base)[((size_t)kernel * kTraceCtas + blockIdx.x +
                                               blockIdx.y * gridDim.x) * kTracePoints + i] = t;
   }
+}
+
+// A plain value (not a time) in a trace slot, e.g. how many items a CTA processed.
+__device__ __forceinline__ void trace_value(const unsigned long long* tr_base, int kernel, int i,
+                                            unsigned long long v) {
+  if (tr_base && threadIdx.x == 0 && blockIdx.x + blockIdx.y * gridDim.x < kTraceCtas)
+    const_cast<unsigned long long*>(tr_base)[((size_t)kernel * kTraceCtas + blockIdx.x +
+                                              blockIdx.y * gridDim.x) * kTracePoints + i] = v;
 }
 
 // Slot table in shared memory as int4 {expert | kind << 16, T, q0, item0}.
@@ -140,9 +149,14 @@ __device__ __forceinline__ int ld_cg(const int* p) { return __ldcg(p); }
 __device__ __forceinline__ unsigned ld_cg(const unsigned* p) { return __ldcg(p); }
 __device__ __forceinline__ float ld_cg(const float* p) { return __ldcg(p); }
 
-// fp32 vector reduction into global memory (sm_90+)
+// fp32 vector reductions into global memory (sm_90+); v4 needs a 16-byte aligned address
 __device__ __forceinline__ void red_add_v2(float* p, float a, float b) {
   asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(a), "f"(b) : "memory");
+}
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
 }
 
 // ---------------------------------------------------------------------------------------------

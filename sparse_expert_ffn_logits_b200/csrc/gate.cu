@@ -42,8 +42,11 @@ struct GateMeta {
   int n0;                     // first neuron
   int key;                    // token tile id (slot * 1024 + tile)
   int xb, xpar, xlast;        // generic variant: token tile buffer, fill phase, last user
+  int end;                    // 1: no more items (the CTA's loops end here)
   int tok[kTileTok];          // register variant: token of each tile column (-1 past the end)
 };
+
+constexpr int kGateChunk = 2;  // items claimed at a time from the work counter
 
 template <int NK, int BPW>
 __global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, Ring rc) {
@@ -88,78 +91,100 @@ __global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, 
   const int n_items = ld_cg(&p.meta[kMetaGateItems]);
   load_slot_table(p, n_slots, s_tab);
   __syncthreads();
-  const int i0 = (int)((long long)blockIdx.x * n_items / gridDim.x);
-  const int i1 = (int)((long long)(blockIdx.x + 1) * n_items / gridDim.x);
   const int H = p.H;
   volatile int* abort = &s_abort;
 
   if (warp == kMetaWarp) {
-    // ---------------- meta: item records (and, generic variant, token tiles) ahead of everyone
+    // ---------------- meta: claims items (its own contiguous share first, then a few at a time
+    // from the work counter, so that fast CTAs take more of the tail), publishes their records one item ahead of the copier and the consumers,
+    // and (generic variant) fills the token tiles.  A record with end = 1 closes the stream.
     int xuse[2] = {0, 0};
-    if (i0 < i1) {
-      int j = find_item_slot(s_tab, n_slots, i0);
-      int I = (s_tab[j].x >> 16) ? p.Ish : p.I;
-      int local = i0 - s_tab[j].w;
-      int tt = local / (I / kTileRows), rg = local % (I / kTileRows);
-      int key = -1, xb = rc.nxb - 1, tok_l = -1;
-      for (int item = i0, mi = 0; item < i1; ++item, ++mi) {
-        const int m = mi % kMetaRing;
-        if (!mbar_wait(&mempty[m], ((mi / kMetaRing) & 1) ^ 1, abort, p.err)) break;
-        const int4 sl = s_tab[j];
-        const int kind = sl.x >> 16, ex = sl.x & 0xffff, T = sl.y, q0 = sl.z;
-        const int nt = min(kTileTok, T - tt * kTileTok);
-        int xpar = 0;
-        if (j * 1024 + tt != key) {
-          key = j * 1024 + tt;
-          tok_l = lane < nt ? __ldcg(&p.pair_token[q0 + tt * kTileTok + lane]) : -1;
-          if constexpr (!kReg) {
-            xb = (xb + 1) % rc.nxb;
-            if (!mbar_wait(&xempty[xb], (xuse[xb] & 1) ^ 1, abort, p.err)) break;
-            xpar = xuse[xb] & 1;
-            xuse[xb]++;
-            if (lane == 0) mbar_arrive_expect_tx(&xfull[xb], kTileTok * H * 2);
-            __syncwarp();
-            if (lane < kTileTok) {
-              const void* src = tok_l >= 0 ? static_cast<const void*>(
-                                                 static_cast<const __nv_bfloat16*>(p.x) +
-                                                 (size_t)tok_l * H)
-                                           : p.zero_row;
-              bulk_g2s(xbuf + xb * rc.xs_bytes + lane * rc.xs_stride, src, H * 2, &xfull[xb]);
-            }
+    // a contiguous share of 7/8 of the items (token tiles stay together), then the rest from
+    // the counter in small chunks
+    const int share = n_items * 7 / 8 / (int)gridDim.x;
+    const int dyn0 = share * (int)gridDim.x;
+    int cb = blockIdx.x * share, ce = cb + share;
+    auto claim = [&]() -> int {
+      if (cb >= ce) {
+        int b = 0;
+        if (lane == 0) b = dyn0 + (int)atomicAdd(&p.claim[0], (unsigned)kGateChunk);
+        b = __shfl_sync(0xffffffffu, b, 0);
+        if (b >= n_items) {
+          cb = ce = n_items;
+          return -1;
+        }
+        cb = b;
+        ce = min(b + kGateChunk, n_items);
+      }
+      return cb++;
+    };
+    auto tile_key = [&](int item) -> int {
+      const int j = find_item_slot(s_tab, n_slots, item);
+      const int I = (s_tab[j].x >> 16) ? p.Ish : p.I;
+      return j * 1024 + (item - s_tab[j].w) / (I / kTileRows);
+    };
+    int key = -1, xb = rc.nxb - 1, tok_l = -1, mi = 0;
+    int cur = claim();
+    int cur_key = cur >= 0 ? tile_key(cur) : -1;
+    for (; cur >= 0 && !*abort; ++mi) {
+      const int nxt = claim();
+      const int nxt_key = nxt >= 0 ? tile_key(nxt) : -1;
+      const int m = mi % kMetaRing;
+      if (!mbar_wait(&mempty[m], ((mi / kMetaRing) & 1) ^ 1, abort, p.err)) break;
+      const int j = find_item_slot(s_tab, n_slots, cur);
+      const int4 sl = s_tab[j];
+      const int kind = sl.x >> 16, ex = sl.x & 0xffff, T = sl.y, q0 = sl.z;
+      const int I = kind ? p.Ish : p.I;
+      const int local = cur - sl.w, tt = local / (I / kTileRows), rg = local % (I / kTileRows);
+      const int nt = min(kTileTok, T - tt * kTileTok);
+      int xpar = 0;
+      if (cur_key != key) {
+        key = cur_key;
+        tok_l = lane < nt ? __ldcg(&p.pair_token[q0 + tt * kTileTok + lane]) : -1;
+        if constexpr (!kReg) {
+          xb = (xb + 1) % rc.nxb;
+          if (!mbar_wait(&xempty[xb], (xuse[xb] & 1) ^ 1, abort, p.err)) break;
+          xpar = xuse[xb] & 1;
+          xuse[xb]++;
+          if (lane == 0) mbar_arrive_expect_tx(&xfull[xb], kTileTok * H * 2);
+          __syncwarp();
+          if (lane < kTileTok) {
+            const void* src = tok_l >= 0 ? static_cast<const void*>(
+                                               static_cast<const __nv_bfloat16*>(p.x) +
+                                               (size_t)tok_l * H)
+                                         : p.zero_row;
+            bulk_g2s(xbuf + xb * rc.xs_bytes + lane * rc.xs_stride, src, H * 2, &xfull[xb]);
           }
-        } else if constexpr (!kReg) {
-          xpar = (xuse[xb] - 1) & 1;
         }
-        // the next item, to know whether this one is the last on its token tile
-        int nj = j, ntt = tt, nrg = rg + 1;
-        if (nrg == I / kTileRows) {
-          nrg = 0;
-          ++ntt;
-          if (ntt * kTileTok >= T) {
-            ntt = 0;
-            ++nj;
-          }
-        }
-        if (lane < kTileTok) s_meta[m].tok[lane] = tok_l;
-        if (lane == 0) {
-          const __nv_bfloat16* base =
-              kind == 0 ? static_cast<const __nv_bfloat16*>(p.gate_r) + (size_t)ex * p.I * H
-                        : static_cast<const __nv_bfloat16*>(p.gate_s) + (size_t)ex * p.Ish * H;
-          s_meta[m].rows = base + (size_t)rg * kTileRows * H;
-          s_meta[m].q0 = q0 + tt * kTileTok;
-          s_meta[m].nt = nt;
-          s_meta[m].n0 = rg * kTileRows;
-          s_meta[m].key = key;
-          s_meta[m].xb = xb;
-          s_meta[m].xpar = xpar;
-          s_meta[m].xlast = item + 1 == i1 || nj * 1024 + ntt != key;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&mfull[m]);
-        if (nj != j && nj < n_slots) I = (s_tab[nj].x >> 16) ? p.Ish : p.I;
-        j = nj;
-        tt = ntt;
-        rg = nrg;
+      } else if constexpr (!kReg) {
+        xpar = (xuse[xb] - 1) & 1;
+      }
+      if (lane < kTileTok) s_meta[m].tok[lane] = tok_l;
+      if (lane == 0) {
+        const __nv_bfloat16* base =
+            kind == 0 ? static_cast<const __nv_bfloat16*>(p.gate_r) + (size_t)ex * p.I * H
+                      : static_cast<const __nv_bfloat16*>(p.gate_s) + (size_t)ex * p.Ish * H;
+        s_meta[m].rows = base + (size_t)rg * kTileRows * H;
+        s_meta[m].q0 = q0 + tt * kTileTok;
+        s_meta[m].nt = nt;
+        s_meta[m].n0 = rg * kTileRows;
+        s_meta[m].key = key;
+        s_meta[m].xb = xb;
+        s_meta[m].xpar = xpar;
+        s_meta[m].xlast = nxt_key != key;
+        s_meta[m].end = 0;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&mfull[m]);
+      cur = nxt;
+      cur_key = nxt_key;
+    }
+    {  // closing record
+      const int m = mi % kMetaRing;
+      mbar_wait(&mempty[m], ((mi / kMetaRing) & 1) ^ 1, abort, p.err);
+      if (lane == 0) {
+        s_meta[m].end = 1;
+        mbar_arrive(&mfull[m]);
       }
     }
     // no token-tile copy may still be landing in shared memory when the CTA exits
@@ -172,9 +197,10 @@ __global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, 
     // ---------------- copier: the item's 16 rows, kc columns per stage, one bulk copy per row
     const uint32_t piece = rc.kc * 2;
     int it = 0;
-    for (int item = i0, mi = 0; item < i1 && !*abort; ++item, ++mi) {
+    for (int mi = 0; !*abort; ++mi) {
       const int m = mi % kMetaRing;
       if (!mbar_wait(&mfull[m], (mi / kMetaRing) & 1, abort, p.err)) break;
+      if (s_meta[m].end) break;
       const __nv_bfloat16* row = s_meta[m].rows + (size_t)(lane & 15) * H;
       __syncwarp();
       if (lane == 0) mbar_arrive(&mempty[m]);
@@ -199,9 +225,16 @@ __global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, 
   bool nan_seen = false;
   const int nblk = rc.kc / 32;
   const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(p.x);
-  for (int item = i0, mi = 0; item < i1; ++item, ++mi) {
+  for (int mi = 0;; ++mi) {
     const int m = mi % kMetaRing;
     mbar_wait(&mfull[m], (mi / kMetaRing) & 1, abort, p.err);
+    // the end (or an abort) is decided by all consumer warps together
+    if (consumer_sync_or(kThreads, s_meta[m].end || *abort)) {
+      trace_value(p.trace, 1, 5, (unsigned long long)mi);
+      break;
+    }
+    if (mi == 0) trace_point(p.trace, 1, 2);
+    trace_point(p.trace, 1, 6);
     const int q0 = s_meta[m].q0, nt = s_meta[m].nt, n0 = s_meta[m].n0, key = s_meta[m].key;
     const int xb = min(max(s_meta[m].xb, 0), max(rc.nxb - 1, 0));  // trusted only w/o abort
     const int xlast = s_meta[m].xlast;
@@ -229,6 +262,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, 
       for (int kc = 0; kc < kXR; ++kc, ++it) {
         const int st = it % rc.ns;
         mbar_wait(&full[st], (it / rc.ns) & 1, abort, p.err);
+        if (it == 0) trace_point(p.trace, 1, 3);
         const unsigned char* stage = ring + (size_t)st * rc.stage_bytes;
 #pragma unroll
         for (int i = 0; i < kXB; ++i) {
@@ -282,6 +316,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, 
         p.act[(size_t)(q0 + ti) * p.Imax + n0 + (ln >> 2) + (c >> 1) * 8] = a;
       }
     }
+    if (mi == 0) trace_point(p.trace, 1, 4);
     ib ^= 1;
   }
   if (nan_seen) set_error(p.err, kErrNanAct);

@@ -100,20 +100,28 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
           for (int i = 0; i < 8; ++i) hist[warp * 8 + i] = (int)c[i];
         }
         __syncthreads();
-        if (threadIdx.x == 0) {
-          int above = 0, digit = 0;
-          for (int d = 15; d >= 0; --d) {
-            int cnt = 0;
+        if (warp == 0) {
+          // lane l < 16 holds digit 15 - l; a suffix scan over the lanes finds the digit
+          int cnt = 0;
+          if (lane < 16) {
+            const int d = 15 - lane;
+#pragma unroll
             for (int w = 0; w < kSelWarps; ++w)
               cnt += (int)(((uint32_t)hist[w * 8 + (d >> 1)] >> ((d & 1) * 16)) & 0xFFFFu);
-            if (above + cnt >= krem) {
-              digit = d;
-              break;
-            }
-            above += cnt;
           }
-          s_digit = digit;
-          s_above = above;
+          int incl = cnt;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+          }
+          const int above = incl - cnt;
+          const unsigned hit = __ballot_sync(0xffffffffu, lane < 16 && above < krem && incl >= krem);
+          const int src = __ffs(hit) - 1;
+          if (lane == src) {
+            s_digit = 15 - lane;
+            s_above = above;
+          }
         }
         __syncthreads();
         krem -= s_above;

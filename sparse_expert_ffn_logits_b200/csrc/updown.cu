@@ -8,7 +8,8 @@
 // lacks the neuron get coefficient 0.
 //
 // Work item = (slot, token tile of 8 pairs, 16 union rows), ordered slot, token tile, rows;
-// each CTA takes a contiguous range of items.  Per item:
+// each CTA takes a contiguous share of the items, then claims the rest one at a time from a
+// counter.  Per item:
 //   1. u[r][c] = W_up[n_r] . x_c           tensor cores, warps split H
 //   2. hc[r][c] = mask * SiLU(g) * u        fp32, rounded to bf16 for the tensor cores
 //   3. y[h][c] = sum_r W_down[h][n_r] hc    tensor cores, 64 h per warp step
@@ -84,7 +85,11 @@ struct UdMeta {
   float w[kTileTok];        // routing weight of each tile column
   int key;                  // token tile id (slot * 1024 + tile)
   int xb, xpar, xlast;      // generic variant: token tile buffer, fill phase, last user
+  int j, tt, rg;            // the item: slot, token tile, row group (for the coefficient warps)
+  int end;                  // 1: no more items (the CTA's loops end here)
 };
+
+constexpr int kUdChunk = 1;  // items claimed at a time from the work counter
 
 template <int NK, int BPW>
 __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p, Ring rc) {
@@ -103,6 +108,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
   uint64_t* mempty = mfull + kMetaRing;
   uint64_t* xfull = mempty + kMetaRing;
   uint64_t* xempty = xfull + 2;
+  uint64_t* mhead = xempty + 2;  // the lead warp has written the record's item
   float(*red)[kWarps][4][32] = reinterpret_cast<float(*)[kWarps][4][32]>(smem + kBarBytes);
   unsigned char* xbuf = smem + kBarBytes + kRedBytes;
   unsigned char* ring = xbuf + rc.nxb * rc.xs_bytes;
@@ -116,6 +122,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
     for (int i = 0; i < kMetaRing; ++i) {
       mbar_init(&mfull[i], 2);  // lead meta warp + the coefficient warp of that record
       mbar_init(&mempty[i], kWarps + 1);
+      mbar_init(&mhead[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&xfull[i], 1);
@@ -154,120 +161,160 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
     __syncthreads();
   }
   const int n_items = s_total;
-  const int i0 = (int)((long long)blockIdx.x * n_items / gridDim.x);
-  const int i1 = (int)((long long)(blockIdx.x + 1) * n_items / gridDim.x);
   const int H = p.H, Imax = p.Imax, Wmax = p.Imax / 32;
   volatile int* abort = &s_abort;
 
-  if (warp >= kMetaWarp) {
-    // ---------------- meta warps: walk the items ahead of the copier and the consumers.
-    // The lead warp owns the token tiles (and the record fields ud, xb, xpar, xlast); coefficient
-    // warp c owns rows, coef, tok and w of the records mi with mi % kCoefWarps == c.
-    const bool lead = warp == kMetaWarp;
-    const int cw = warp - kCoefWarp0;
+  if (warp == kMetaWarp) {
+    // ---------------- lead meta warp: claims items (its own contiguous share of 3/4 of them
+    // first, then one at a time from the work counter, so that fast CTAs take more of the tail),
+    // owns the token tiles and the record fields ud, key, xb, xpar, xlast; publishes the item
+    // (mhead) for the coefficient warp of the record.  Two records with end = 1 close the
+    // stream: one for the copier and consumers, one more so that both coefficient warps see it.
     int xuse[2] = {0, 0};
-    if (i0 < i1) {
-      int j = find_item_slot(s_tab, n_slots, i0);
-      int nrg = (s_ucnt[j] + kTileRows - 1) / kTileRows;
-      int local = i0 - s_tab[j].w;
-      int tt = local / nrg, rg = local % nrg;
-      int key = -1, xb = rc.nxb - 1;
-      for (int item = i0, mi = 0; item < i1; ++item, ++mi) {
-        const int m = mi % kMetaRing;
-        const int4 sl = s_tab[j];
-        const int kind = sl.x >> 16, ex = sl.x & 0xffff, T = sl.y, q0 = sl.z, rows = s_ucnt[j];
-        const int nt = min(kTileTok, T - tt * kTileTok);
-        const int qt = q0 + tt * kTileTok;
-        // the next item, to know whether this one is the last on its token tile
-        int nj = j, ntt = tt, nrg2 = rg + 1;
-        if (nrg2 >= nrg) {
-          nrg2 = 0;
-          ++ntt;
-          if (ntt * kTileTok >= T) {
-            ntt = 0;
-            ++nj;
-            while (nj < n_slots && s_ucnt[nj] == 0) ++nj;
-          }
+    const int share = n_items * 3 / 4 / (int)gridDim.x;
+    const int dyn0 = share * (int)gridDim.x;
+    int cb = blockIdx.x * share, ce = cb + share;
+    auto claim = [&]() -> int {
+      if (cb >= ce) {
+        int b = 0;
+        if (lane == 0) b = dyn0 + (int)atomicAdd(&p.claim[1], (unsigned)kUdChunk);
+        b = __shfl_sync(0xffffffffu, b, 0);
+        if (b >= n_items) {
+          cb = ce = n_items;
+          return -1;
         }
-        const bool mine = lead || mi % kCoefWarps == cw;
-        if (mine) {
-          if (!mbar_wait(&mempty[m], ((mi / kMetaRing) & 1) ^ 1, abort, p.err)) break;
-        }
-        if (lead) {
-          int xpar = 0;
-          if (j * 1024 + tt != key) {
-            key = j * 1024 + tt;
-            if constexpr (!kReg) {
-              xb = (xb + 1) % rc.nxb;
-              if (!mbar_wait(&xempty[xb], (xuse[xb] & 1) ^ 1, abort, p.err)) break;
-              xpar = xuse[xb] & 1;
-              xuse[xb]++;
-              const int tok_l = lane < nt ? __ldcg(&p.pair_token[qt + lane]) : -1;
-              if (lane == 0) mbar_arrive_expect_tx(&xfull[xb], kTileTok * H * 2);
-              __syncwarp();
-              if (lane < kTileTok) {
-                const void* src = tok_l >= 0 ? static_cast<const void*>(
-                                                   static_cast<const __nv_bfloat16*>(p.x) +
-                                                   (size_t)tok_l * H)
-                                             : p.zero_row;
-                bulk_g2s(xbuf + xb * rc.xs_bytes + lane * rc.xs_stride, src, H * 2, &xfull[xb]);
-              }
-            }
-          } else if constexpr (!kReg) {
-            xpar = (xuse[xb] - 1) & 1;
-          }
-          if (lane == 0) {
-            s_meta[m].ud = kind == 0 ? static_cast<const __nv_bfloat16*>(p.updown_r) +
-                                           (size_t)ex * p.I * 2 * H
-                                     : static_cast<const __nv_bfloat16*>(p.updown_s) +
-                                           (size_t)ex * p.Ish * 2 * H;
-            s_meta[m].key = key;
-            s_meta[m].xb = xb;
-            s_meta[m].xpar = xpar;
-            s_meta[m].xlast = item + 1 == i1 || nj * 1024 + ntt != key;
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&mfull[m]);
-        } else if (mine) {
-          // row of this lane (lanes 0..15) and token of this lane (lanes 0..7)
-          const int ridx = rg * kTileRows + (lane & 15);
-          const int n_l =
-              __ldcg(&p.ulist[(size_t)j * Imax + (ridx < rows ? ridx : rg * kTileRows)]);
-          const int tok_l = lane < nt ? __ldcg(&p.pair_token[qt + lane]) : -1;
-          const float w_l = lane < nt ? __ldcg(&p.pair_w[qt + lane]) : 0.f;
-          // coefficients: lane l covers row l/2, columns 4*(l&1) .. +3
-          const int r = lane >> 1, c0 = (lane & 1) * 4;
-          const int n = __shfl_sync(0xffffffffu, n_l, r);
-          const bool rvalid = rg * kTileRows + r < rows;
-          uint32_t bits[4];
-          float av[4];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int q = qt + c0 + c;
-            const bool ok = rvalid && c0 + c < nt;
-            bits[c] = ok ? __ldcg(&p.maskbits[(size_t)q * Wmax + (n >> 5)]) : 0u;
-            av[c] = ok ? __ldcg(&p.act[(size_t)q * Imax + n]) : 0.f;
-          }
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            s_meta[m].coef[r][c0 + c] = ((bits[c] >> (n & 31)) & 1u) ? av[c] : 0.f;
-          if (lane < kTileRows) s_meta[m].rows[lane] = n_l;
-          if (lane < kTileTok) {
-            s_meta[m].tok[lane] = tok_l;
-            s_meta[m].w[lane] = w_l;
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&mfull[m]);
-        }
-        if (nj != j && nj < n_slots) nrg = (s_ucnt[nj] + kTileRows - 1) / kTileRows;
-        j = nj;
-        tt = ntt;
-        rg = nrg2;
+        cb = b;
+        ce = min(b + kUdChunk, n_items);
       }
+      return cb++;
+    };
+    struct Pos {
+      int j, tt, rg;
+    };
+    auto decode = [&](int item) -> Pos {
+      Pos d;
+      d.j = find_item_slot(s_tab, n_slots, item);
+      const int nrg = (s_ucnt[d.j] + kTileRows - 1) / kTileRows;
+      const int local = item - s_tab[d.j].w;
+      d.tt = local / nrg;
+      d.rg = local % nrg;
+      return d;
+    };
+    int key = -1, xb = rc.nxb - 1, mi = 0;
+    int cur = claim();
+    Pos cp = cur >= 0 ? decode(cur) : Pos{0, 0, 0};
+    for (; cur >= 0 && !*abort; ++mi) {
+      const int nxt = claim();
+      const Pos np = nxt >= 0 ? decode(nxt) : Pos{0, 0, 0};
+      const int nxt_key = nxt >= 0 ? np.j * 1024 + np.tt : -1;
+      const int m = mi % kMetaRing;
+      if (!mbar_wait(&mempty[m], ((mi / kMetaRing) & 1) ^ 1, abort, p.err)) break;
+      const int4 sl = s_tab[cp.j];
+      const int kind = sl.x >> 16, ex = sl.x & 0xffff, T = sl.y, q0 = sl.z;
+      const int nt = min(kTileTok, T - cp.tt * kTileTok);
+      const int qt = q0 + cp.tt * kTileTok;
+      int xpar = 0;
+      if (cp.j * 1024 + cp.tt != key) {
+        key = cp.j * 1024 + cp.tt;
+        if constexpr (!kReg) {
+          xb = (xb + 1) % rc.nxb;
+          if (!mbar_wait(&xempty[xb], (xuse[xb] & 1) ^ 1, abort, p.err)) break;
+          xpar = xuse[xb] & 1;
+          xuse[xb]++;
+          const int tok_l = lane < nt ? __ldcg(&p.pair_token[qt + lane]) : -1;
+          if (lane == 0) mbar_arrive_expect_tx(&xfull[xb], kTileTok * H * 2);
+          __syncwarp();
+          if (lane < kTileTok) {
+            const void* src = tok_l >= 0 ? static_cast<const void*>(
+                                               static_cast<const __nv_bfloat16*>(p.x) +
+                                               (size_t)tok_l * H)
+                                         : p.zero_row;
+            bulk_g2s(xbuf + xb * rc.xs_bytes + lane * rc.xs_stride, src, H * 2, &xfull[xb]);
+          }
+        }
+      } else if constexpr (!kReg) {
+        xpar = (xuse[xb] - 1) & 1;
+      }
+      if (lane == 0) {
+        s_meta[m].ud = kind == 0 ? static_cast<const __nv_bfloat16*>(p.updown_r) +
+                                       (size_t)ex * p.I * 2 * H
+                                 : static_cast<const __nv_bfloat16*>(p.updown_s) +
+                                       (size_t)ex * p.Ish * 2 * H;
+        s_meta[m].key = key;
+        s_meta[m].xb = xb;
+        s_meta[m].xpar = xpar;
+        s_meta[m].xlast = nxt_key != key;
+        s_meta[m].j = cp.j;
+        s_meta[m].tt = cp.tt;
+        s_meta[m].rg = cp.rg;
+        s_meta[m].end = 0;
+        mbar_arrive(&mhead[m]);
+        mbar_arrive(&mfull[m]);
+      }
+      __syncwarp();
+      cur = nxt;
+      cp = np;
     }
-    if (lead)
-      for (int b = 0; b < rc.nxb; ++b)
-        if (xuse[b] > 0) mbar_drain(&xfull[b], (xuse[b] - 1) & 1);
+    for (int e = 0; e < 2; ++e, ++mi) {  // closing records
+      const int m = mi % kMetaRing;
+      mbar_wait(&mempty[m], ((mi / kMetaRing) & 1) ^ 1, abort, p.err);
+      if (lane == 0) {
+        s_meta[m].end = 1;
+        mbar_arrive(&mhead[m]);
+        mbar_arrive(&mfull[m]);
+      }
+      __syncwarp();
+    }
+    for (int b = 0; b < rc.nxb; ++b)
+      if (xuse[b] > 0) mbar_drain(&xfull[b], (xuse[b] - 1) & 1);
+    return;
+  }
+
+  if (warp >= kCoefWarp0) {
+    // ---------------- coefficient warp c: rows, coef, tok and w of the records mi with
+    // mi % kCoefWarps == c (so it always uses the same meta slots)
+    const int cw = warp - kCoefWarp0;
+    for (int mi = cw;; mi += kCoefWarps) {
+      const int m = mi % kMetaRing;
+      if (!mbar_wait(&mhead[m], (mi / kMetaRing) & 1, abort, p.err)) break;
+      if (s_meta[m].end) {
+        if (lane == 0) mbar_arrive(&mfull[m]);
+        break;
+      }
+      const int j = s_meta[m].j, tt = s_meta[m].tt, rg = s_meta[m].rg;
+      const int4 sl = s_tab[j];
+      const int T = sl.y, q0 = sl.z, rows = s_ucnt[j];
+      const int nt = min(kTileTok, T - tt * kTileTok);
+      const int qt = q0 + tt * kTileTok;
+      // row of this lane (lanes 0..15) and token of this lane (lanes 0..7)
+      const int ridx = rg * kTileRows + (lane & 15);
+      const int n_l = __ldcg(&p.ulist[(size_t)j * Imax + (ridx < rows ? ridx : rg * kTileRows)]);
+      const int tok_l = lane < nt ? __ldcg(&p.pair_token[qt + lane]) : -1;
+      const float w_l = lane < nt ? __ldcg(&p.pair_w[qt + lane]) : 0.f;
+      // coefficients: lane l covers row l/2, columns 4*(l&1) .. +3
+      const int r = lane >> 1, c0 = (lane & 1) * 4;
+      const int n = __shfl_sync(0xffffffffu, n_l, r);
+      const bool rvalid = rg * kTileRows + r < rows;
+      uint32_t bits[4];
+      float av[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int q = qt + c0 + c;
+        const bool ok = rvalid && c0 + c < nt;
+        bits[c] = ok ? __ldcg(&p.maskbits[(size_t)q * Wmax + (n >> 5)]) : 0u;
+        av[c] = ok ? __ldcg(&p.act[(size_t)q * Imax + n]) : 0.f;
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        s_meta[m].coef[r][c0 + c] = ((bits[c] >> (n & 31)) & 1u) ? av[c] : 0.f;
+      if (lane < kTileRows) s_meta[m].rows[lane] = n_l;
+      if (lane < kTileTok) {
+        s_meta[m].tok[lane] = tok_l;
+        s_meta[m].w[lane] = w_l;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&mfull[m]);
+    }
     return;
   }
 
@@ -275,9 +322,10 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
     // ---------------- copier: up pieces, then down pieces, of the item's 16 rows
     const uint32_t piece = rc.kc * 2;
     int it = 0;
-    for (int item = i0, mi = 0; item < i1 && !*abort; ++item, ++mi) {
+    for (int mi = 0; !*abort; ++mi) {
       const int m = mi % kMetaRing;
       if (!mbar_wait(&mfull[m], (mi / kMetaRing) & 1, abort, p.err)) break;
+      if (s_meta[m].end) break;
       const __nv_bfloat16* row = s_meta[m].ud + (size_t)s_meta[m].rows[lane & 15] * 2 * H;
       __syncwarp();
       if (lane == 0) mbar_arrive(&mempty[m]);
@@ -308,9 +356,16 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
   int it = 0, ib = 0, cur = -1;
   const int nblk = rc.kc / 32, nsub = rc.kc / 64;
   const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(p.x);
-  for (int item = i0, mi = 0; item < i1; ++item, ++mi) {
+  for (int mi = 0;; ++mi) {
     const int m = mi % kMetaRing;
     mbar_wait(&mfull[m], (mi / kMetaRing) & 1, abort, p.err);
+    // the end (or an abort) is decided by all consumer warps together
+    if (consumer_sync_or(kThreads, s_meta[m].end || *abort)) {
+      trace_value(p.trace, 3, 5, (unsigned long long)mi);
+      break;
+    }
+    if (mi == 0) trace_point(p.trace, 3, 2);
+    trace_point(p.trace, 3, 6);
     const UdMeta& mt = s_meta[m];
     const int xb = min(max(mt.xb, 0), max(rc.nxb - 1, 0));  // a record is trusted only w/o abort
     const int xlast = mt.xlast;
@@ -341,6 +396,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
       for (int kc = 0; kc < kXR; ++kc, ++it) {
         const int st = it % rc.ns;
         mbar_wait(&full[st], (it / rc.ns) & 1, abort, p.err);
+        if (it == 0) trace_point(p.trace, 3, 3);
         const unsigned char* stage = ring + (size_t)st * rc.stage_bytes;
 #pragma unroll
         for (int i = 0; i < kXB; ++i) {
@@ -405,22 +461,31 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
         const uint32_t w0v[4] = {r0.x, r0.y, r0.z, r0.w}, w1v[4] = {r1.x, r1.y, r1.z, r1.w};
         const uint32_t w2v[4] = {r2.x, r2.y, r2.z, r2.w}, w3v[4] = {r3.x, r3.y, r3.z, r3.w};
         const int hb = kc * rc.kc + sc * 64 + 8 * g;
+        // mma i gives h = hb + 2i, 2i + 1 for the thread's two tokens: eight consecutive h per
+        // token, reduced as two 16-byte vectors (the L2 reductions are the costly part here)
+        float acc[4][4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          float acc[4] = {0.f, 0.f, 0.f, 0.f};
-          mma_16816(acc, __byte_perm(w0v[i], w1v[i], 0x5410), __byte_perm(w0v[i], w1v[i], 0x7632),
-                    __byte_perm(w2v[i], w3v[i], 0x5410), __byte_perm(w2v[i], w3v[i], 0x7632), b0,
-                    b1);
-          const int h = hb + 2 * i;
-          if (!aborted && tok0 >= 0)
-            red_add_v2(p.out_acc + (size_t)tok0 * H + h, w0 * acc[0], w0 * acc[2]);
-          if (!aborted && tok1 >= 0)
-            red_add_v2(p.out_acc + (size_t)tok1 * H + h, w1 * acc[1], w1 * acc[3]);
+          acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+          mma_16816(acc[i], __byte_perm(w0v[i], w1v[i], 0x5410),
+                    __byte_perm(w0v[i], w1v[i], 0x7632), __byte_perm(w2v[i], w3v[i], 0x5410),
+                    __byte_perm(w2v[i], w3v[i], 0x7632), b0, b1);
+        }
+        if (!aborted && tok0 >= 0) {
+          float* o = p.out_acc + (size_t)tok0 * H + hb;
+          red_add_v4(o, w0 * acc[0][0], w0 * acc[0][2], w0 * acc[1][0], w0 * acc[1][2]);
+          red_add_v4(o + 4, w0 * acc[2][0], w0 * acc[2][2], w0 * acc[3][0], w0 * acc[3][2]);
+        }
+        if (!aborted && tok1 >= 0) {
+          float* o = p.out_acc + (size_t)tok1 * H + hb;
+          red_add_v4(o, w1 * acc[0][1], w1 * acc[0][3], w1 * acc[1][1], w1 * acc[1][3]);
+          red_add_v4(o + 4, w1 * acc[2][1], w1 * acc[2][3], w1 * acc[3][1], w1 * acc[3][3]);
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);
     }
+    if (mi == 0) trace_point(p.trace, 3, 4);
     ib ^= 1;
   }
   trace_point(p.trace, 3, 7);
