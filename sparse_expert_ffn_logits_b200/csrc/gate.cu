@@ -376,9 +376,8 @@ __global__ void __launch_bounds__(kThreads) gate_f32_kernel(FwdParams p) {
 }
 
 template <int NK, int BPW>
-cudaError_t set_gate_smem(const Ring& r) {
-  return cudaFuncSetAttribute(gate_tma_kernel<NK, BPW>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, r.smem_bytes);
+cudaError_t set_gate_smem(int budget) {
+  return allow_max_smem(gate_tma_kernel<NK, BPW>, budget);
 }
 
 template <int NK, int BPW>
@@ -473,11 +472,11 @@ cudaError_t configure_gate(int dtype, int H, int smem_budget, LaunchShape* ls) {
   if (ls->ring_gate.ns < 2) return cudaErrorInvalidConfiguration;
   ls->grid_gate = ls->nsm;
   switch (ls->variant) {
-    case 1: return set_gate_smem<1, 2>(ls->ring_gate);
-    case 2: return set_gate_smem<1, 8>(ls->ring_gate);
-    case 3: return set_gate_smem<3, 4>(ls->ring_gate);
-    case 4: return set_gate_smem<4, 5>(ls->ring_gate);
-    default: return set_gate_smem<0, 0>(ls->ring_gate);
+    case 1: return set_gate_smem<1, 2>(smem_budget);
+    case 2: return set_gate_smem<1, 8>(smem_budget);
+    case 3: return set_gate_smem<3, 4>(smem_budget);
+    case 4: return set_gate_smem<4, 5>(smem_budget);
+    default: return set_gate_smem<0, 0>(smem_budget);
   }
 }
 

@@ -59,4 +59,16 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
+// Lets a kernel use all the dynamic shared memory the device allows next to its static shared
+// memory.  The attribute is per kernel and per device, so it is always set to this maximum:
+// a handle with smaller sizes must never lower the limit under another live handle.
+template <typename... KArgs>
+cudaError_t allow_max_smem(void (*kernel)(KArgs...), int optin_budget) {
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              optin_budget - (int)fa.sharedSizeBytes);
+}
+
 }  // namespace moe

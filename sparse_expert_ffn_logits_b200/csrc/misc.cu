@@ -3,8 +3,8 @@
 
 namespace moe {
 
-cudaError_t configure_router(int max_E, int max_B);
-cudaError_t configure_select(int imax, int* occupancy);
+cudaError_t configure_router(int budget);
+cudaError_t configure_select(int imax, int budget, int* occupancy);
 cudaError_t configure_gate(int dtype, int H, int smem_budget, LaunchShape* ls);
 cudaError_t configure_updown(int dtype, int H, int smem_budget, LaunchShape* ls);
 
@@ -111,10 +111,10 @@ cudaError_t configure_kernels(int dtype, int imax, int max_E, int max_B, int H, 
   int budget = 0;
   e = cudaDeviceGetAttribute(&budget, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (e != cudaSuccess) return e;
-  e = configure_router(max_E, max_B);
+  e = configure_router(budget);
   if (e != cudaSuccess) return e;
   int occ_sel = 0;
-  e = configure_select(imax, &occ_sel);
+  e = configure_select(imax, budget, &occ_sel);
   if (e != cudaSuccess) return e;
   ls->grid_select = ls->nsm * (occ_sel > 0 ? occ_sel : 1);
   e = configure_gate(dtype, H, budget, ls);

@@ -361,25 +361,19 @@ cudaError_t launch_router(const FwdParams& p, int dtype, cudaStream_t st) {
 }
 
 template <typename T>
-cudaError_t configure_router_t(int smem) {
-  cudaError_t e = cudaSuccess;
-  e = cudaFuncSetAttribute(router_kernel<T, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(router_kernel<T, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(router_kernel<T, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(router_kernel<T, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(router_kernel<T, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+cudaError_t configure_router_t(int budget) {
+  cudaError_t e = allow_max_smem(router_kernel<T, 1>, budget);
+  if (e == cudaSuccess) e = allow_max_smem(router_kernel<T, 2>, budget);
+  if (e == cudaSuccess) e = allow_max_smem(router_kernel<T, 4>, budget);
+  if (e == cudaSuccess) e = allow_max_smem(router_kernel<T, 8>, budget);
+  if (e == cudaSuccess) e = allow_max_smem(router_kernel<T, 16>, budget);
   return e;
 }
 
-cudaError_t configure_router(int max_E, int max_B) {
-  const int smem = (int)router_smem_bytes(max_E, max_B);
-  cudaError_t e = configure_router_t<__nv_bfloat16>(smem);
+cudaError_t configure_router(int budget) {
+  cudaError_t e = configure_router_t<__nv_bfloat16>(budget);
   if (e != cudaSuccess) return e;
-  return configure_router_t<float>(smem);
+  return configure_router_t<float>(budget);
 }
 
 }  // namespace moe

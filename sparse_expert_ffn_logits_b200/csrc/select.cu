@@ -248,10 +248,9 @@ cudaError_t launch_select(const FwdParams& p, const LaunchShape& ls, cudaStream_
                     pdl, p);
 }
 
-cudaError_t configure_select(int imax, int* occupancy) {
+cudaError_t configure_select(int imax, int budget, int* occupancy) {
   const size_t smem = select_smem_bytes(imax);
-  cudaError_t e =
-      cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = allow_max_smem(select_kernel, budget);
   if (e != cudaSuccess) return e;
   return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occupancy, select_kernel, kSelThreads, smem);
 }

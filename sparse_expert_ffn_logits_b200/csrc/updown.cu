@@ -575,9 +575,8 @@ __global__ void __launch_bounds__(kThreads) updown_f32_kernel(FwdParams p) {
 }  // namespace
 
 template <int NK, int BPW>
-cudaError_t set_ud_smem(const Ring& r) {
-  return cudaFuncSetAttribute(updown_tma_kernel<NK, BPW>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, r.smem_bytes);
+cudaError_t set_ud_smem(int budget) {
+  return allow_max_smem(updown_tma_kernel<NK, BPW>, budget);
 }
 
 template <int NK, int BPW>
@@ -628,11 +627,11 @@ cudaError_t configure_updown(int dtype, int H, int smem_budget, LaunchShape* ls)
   if (ls->ring_ud.ns < 2) return cudaErrorInvalidConfiguration;
   ls->grid_updown = ls->nsm;
   switch (ls->variant) {
-    case 1: return set_ud_smem<1, 2>(ls->ring_ud);
-    case 2: return set_ud_smem<1, 8>(ls->ring_ud);
-    case 3: return set_ud_smem<3, 4>(ls->ring_ud);
-    case 4: return set_ud_smem<4, 5>(ls->ring_ud);
-    default: return set_ud_smem<0, 0>(ls->ring_ud);
+    case 1: return set_ud_smem<1, 2>(smem_budget);
+    case 2: return set_ud_smem<1, 8>(smem_budget);
+    case 3: return set_ud_smem<3, 4>(smem_budget);
+    case 4: return set_ud_smem<4, 5>(smem_budget);
+    default: return set_ud_smem<0, 0>(smem_budget);
   }
 }
 

@@ -141,6 +141,18 @@ def test_olmoe_full_batch(olmoe):
     _run(olmoe, 64, ("topk", 0.9), batch_index=8, expert_cache=cache)
 
 
+def test_second_handle_keeps_first_working(olmoe):
+    """A smaller handle created later must not shrink the kernels' shared-memory limits under
+    the larger one that is still alive."""
+    small = synth.configs.LayerShape("small-bf16", 512, 16, 4, 256, n_shared=1, inter_shared=384)
+    dl = DeviceLayer(small, max_tokens=2)
+    try:
+        _run(dl, 2, ("topk", 0.5))
+        _run(olmoe, 256, ("topk", 0.9), batch_index=9, tokens=np.arange(3, 256, 16))
+    finally:
+        dl.close()
+
+
 # ---------------------------------------------------------------------------------------------
 @pytest.fixture(scope="module")
 def dsv2l():
