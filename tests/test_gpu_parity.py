@@ -147,7 +147,7 @@ def test_second_handle_keeps_first_working(olmoe):
     small = synth.configs.LayerShape("small-bf16", 512, 16, 4, 256, n_shared=1, inter_shared=384)
     dl = DeviceLayer(small, max_tokens=2)
     try:
-        _run(dl, 2, ("topk", 0.5))
+        _run(dl, 2, ("topk", 0.5), ("topk", 0.5))
         _run(olmoe, 256, ("topk", 0.9), batch_index=9, tokens=np.arange(3, 256, 16))
     finally:
         dl.close()
