@@ -173,6 +173,27 @@ moe_status moe_get_error(moe_handle* h, int* device_code);
 /* Frees the workspace and the handle (synchronises the device first).  NULL is a no-op. */
 moe_status moe_destroy(moe_handle* h);
 
+/* Routing only, with no handle and no device allocation.  The paper has no counterpart: its
+ * router runs inside the layer.  This is for callers that need only each token's expert choice
+ * and cannot allocate device memory at that point (for instance a scheduler that plans expert
+ * placement while a caching allocator holds all free memory).  It computes exactly what
+ * moe_forward's router step computes:
+ *   cfg       hidden, n_routed, top_k, dtype and route are read (the other fields are ignored);
+ *             the limits of moe_config apply
+ *   x         [n_tokens][hidden]  device, dtype, 16-byte aligned, read
+ *   router    [n_routed][hidden]  device, dtype, 16-byte aligned, read
+ *   topk_idx  [n_tokens][top_k]   device int32, written: experts by logit descending, ties to
+ *                                 the lower expert index
+ *   topk_w    [n_tokens][top_k]   device fp32, written: the routing weights of cfg->route
+ *   stream    cudaStream_t, or NULL for the default stream; the call is asynchronous
+ * It runs on a 2 MiB scratch area that the library holds per device.  n_tokens <= 256;
+ * n_tokens > 256 is UNSUPPORTED, n_tokens < 0 INVALID_ARG, n_tokens = 0 a no-op.  The first call
+ * on a device sets the scratch area up (it may load the module), so make it before any stream
+ * capture.  Calls that overlap in time on one device share the scratch area and race: serialise
+ * them.  A NaN logit ranks lowest; no device error word is reported. */
+moe_status moe_route_noalloc(const moe_config* cfg, const void* x, int n_tokens,
+                             const void* router, int* topk_idx, float* topk_w, void* stream);
+
 /* Static description of a status code. */
 const char* moe_status_string(moe_status s);
 

@@ -51,7 +51,7 @@ _LIB = None
 # C entry points declared in include/moe.h
 EXPORTS = ("moe_create", "moe_packed_bytes", "moe_pack_experts", "moe_forward",
            "moe_forward_host", "moe_debug_lists", "moe_profile_stages", "moe_read_trace",
-           "moe_get_error", "moe_destroy", "moe_status_string")
+           "moe_get_error", "moe_destroy", "moe_route_noalloc", "moe_status_string")
 MOE_STAGE_EVENTS = 6
 STAGES = ("router", "gate", "select", "updown", "finalize")
 
@@ -78,6 +78,7 @@ def _lib():
         lib.moe_read_trace.argtypes = [P, P, ctypes.c_size_t]
         lib.moe_get_error.argtypes = [P, ctypes.POINTER(I)]
         lib.moe_destroy.argtypes = [P]
+        lib.moe_route_noalloc.argtypes = [ctypes.POINTER(MoEConfig), P, I, P, P, P, P]
         lib.moe_status_string.argtypes = [I]
         lib.moe_status_string.restype = ctypes.c_char_p
         for f in EXPORTS[:-1]:
@@ -206,3 +207,10 @@ def moe_get_error(h):
 
 def moe_destroy(h):
     _check(_lib().moe_destroy(ctypes.c_void_p(h) if h else None), "moe_destroy")
+
+
+def moe_route_noalloc(cfg, x, n_tokens, router, topk_idx, topk_w, stream=None):
+    """Routing only, with no handle and no device allocation (see include/moe.h)."""
+    _check(_lib().moe_route_noalloc(ctypes.byref(cfg), _ptr(x), int(n_tokens), _ptr(router),
+                                    _ptr(topk_idx), _ptr(topk_w), _stream(stream)),
+           "moe_route_noalloc")

@@ -1,0 +1,152 @@
+// route_noalloc.cu - routing only (router logits, top-k experts, routing weights) for one batch,
+// with no handle and no device allocation.
+//
+// Who calls it.  moe_create allocates the whole layer workspace.  Some callers need only the
+// expert choice of each token, and cannot allocate device memory where they ask for it:
+//   - a scheduler that prefetches or places experts from the next batch's routing, running
+//     while a caching allocator has reserved all free device memory (a cudaMalloc there would
+//     fail, or force the allocator to release and fragment its pool);
+//   - code that must not change the device's memory footprint, such as a memory-budgeted
+//     service whose footprint was measured at start-up.
+// For them this entry point runs the router kernel of the layer (logit tiles, top-k, grouping)
+// on a fixed scratch area compiled into the library, instead of a handle's workspace.
+//
+// The scratch area is one static device array per device.  The first call on a device looks up
+// its address (cudaGetSymbolAddress, which may load the module) and sets the router kernels'
+// shared-memory limit.  That first call should therefore come before any stream capture.  Every
+// later call only clears the zero-at-start words and launches.  Calls that overlap in time on one
+// device, from two streams or two threads, share the scratch area and race: the caller
+// serialises them.
+#include <mutex>
+
+#include "../../include/moe.h"
+#include "kernels.h"
+
+namespace moe {
+cudaError_t configure_router(int budget);
+}
+
+namespace {
+
+constexpr size_t kScratchBytes = (size_t)2 << 20;  // 2 MiB: room for 256 tokens x 512 experts
+constexpr int kNoAllocMaxTokens = 256;
+constexpr int kMaxDevices = 64;
+
+// The scratch area (zero at module load; the zero-at-start words are cleared again by every call).
+static __device__ __align__(256) unsigned char g_route_scratch[kScratchBytes];
+
+std::mutex g_setup_mu;
+void* g_scratch_addr[kMaxDevices];  // device address of g_route_scratch per device; null = not set up
+
+// Once per device, with that device current: the scratch area's address and the router
+// kernels' shared-memory limit.  Returns the address, or null (with *err set) on failure.
+void* scratch_for_current_device(cudaError_t* err) {
+  int dev = 0;
+  *err = cudaGetDevice(&dev);
+  if (*err != cudaSuccess) return nullptr;
+  if (dev < 0 || dev >= kMaxDevices) {
+    *err = cudaErrorInvalidDevice;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(g_setup_mu);
+  if (!g_scratch_addr[dev]) {
+    void* ptr = nullptr;
+    *err = cudaGetSymbolAddress(&ptr, g_route_scratch);
+    if (*err != cudaSuccess || !ptr) return nullptr;
+    int budget = 0;
+    *err = cudaDeviceGetAttribute(&budget, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (*err != cudaSuccess) return nullptr;
+    *err = moe::configure_router(budget);
+    if (*err != cudaSuccess) return nullptr;
+    g_scratch_addr[dev] = ptr;
+  }
+  return g_scratch_addr[dev];
+}
+
+size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+}  // namespace
+
+extern "C" moe_status moe_route_noalloc(const moe_config* cfg, const void* x, int n_tokens,
+                                        const void* router, int* topk_idx, float* topk_w,
+                                        void* stream) {
+  if (!cfg) return MOE_ERR_INVALID_ARG;
+  if (cfg->dtype != MOE_BF16 && cfg->dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
+  if (cfg->route < MOE_ROUTE_SOFTMAX_TOPK || cfg->route > MOE_ROUTE_SIGMOID)
+    return MOE_ERR_INVALID_ARG;
+  if (cfg->hidden <= 0 || cfg->n_routed <= 0 || cfg->top_k <= 0 || cfg->top_k > cfg->n_routed)
+    return MOE_ERR_INVALID_ARG;
+  if (cfg->hidden % 64 || cfg->hidden > 8192 || cfg->n_routed > moe::kMaxRouted ||
+      cfg->top_k > moe::kMaxTopK)
+    return MOE_ERR_UNSUPPORTED;
+  if (n_tokens < 0) return MOE_ERR_INVALID_ARG;
+  if (n_tokens > kNoAllocMaxTokens) return MOE_ERR_UNSUPPORTED;  // beyond the scratch area
+  if (n_tokens == 0) return MOE_OK;
+  if (!x || !router || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(router)) & 15u)
+    return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(topk_idx) | reinterpret_cast<uintptr_t>(topk_w)) & 3u)
+    return MOE_ERR_INVALID_ARG;
+
+  const int B = n_tokens, E = cfg->n_routed, k = cfg->top_k, H = cfg->hidden;
+  const int hsplit = moe::router_hsplit(E, B, H);
+  const int tiles = (B + moe::kTileTok - 1) / moe::kTileTok;
+  // scratch layout: everything the router kernel writes, then the words that start at zero
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  const size_t o_logits = take(sizeof(float) * B * E);
+  const size_t o_part = take(sizeof(float) * hsplit * B * E);
+  const size_t o_pidx = take(sizeof(int) * B * k);
+  const size_t o_ptok = take(sizeof(int) * B * k);
+  const size_t o_pw = take(sizeof(float) * B * k);
+  const size_t o_pslot = take(sizeof(int) * B * k);
+  const size_t o_slots = take(sizeof(moe::Slot) * E);
+  const size_t o_meta = take(sizeof(int) * moe::kMetaWords);
+  const size_t o_zero = off;  // tile tickets, the batch ticket and the error word start at zero
+  const size_t o_tick = take(sizeof(unsigned) * tiles);
+  const size_t o_gtick = take(sizeof(unsigned));
+  const size_t o_err = take(sizeof(int));
+  const size_t zero_bytes = off - o_zero;
+  if (off > kScratchBytes) return MOE_ERR_UNSUPPORTED;
+
+  cudaError_t ce = cudaSuccess;
+  char* base = static_cast<char*>(scratch_for_current_device(&ce));
+  if (!base) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(base + o_zero, 0, zero_bytes, st) != cudaSuccess) return MOE_ERR_CUDA;
+
+  moe::FwdParams p = {};
+  p.H = H;
+  p.E = E;
+  p.k = k;
+  p.S = 0;
+  p.I = moe::kTileRows;  // the grouping phase counts gate items; no later kernel reads them
+  p.Ish = moe::kTileRows;
+  p.B = B;
+  p.Imax = moe::kTileRows;
+  p.Bmax = B;
+  p.hsplit = hsplit;
+  p.route = (int)cfg->route;
+  p.x = x;
+  p.router = router;
+  p.logits = reinterpret_cast<float*>(base + o_logits);
+  p.logit_part = reinterpret_cast<float*>(base + o_part);
+  p.topk_idx = topk_idx;
+  p.topk_w = topk_w;
+  p.pair_index = reinterpret_cast<int*>(base + o_pidx);
+  p.pair_token = reinterpret_cast<int*>(base + o_ptok);
+  p.pair_w = reinterpret_cast<float*>(base + o_pw);
+  p.pair_slot = reinterpret_cast<int*>(base + o_pslot);
+  p.slots = reinterpret_cast<moe::Slot*>(base + o_slots);
+  p.meta = reinterpret_cast<int*>(base + o_meta);
+  p.tile_ticket = reinterpret_cast<unsigned*>(base + o_tick);
+  p.global_ticket = reinterpret_cast<unsigned*>(base + o_gtick);
+  p.err = reinterpret_cast<int*>(base + o_err);
+  p.trace = nullptr;
+  return moe::launch_router(p, cfg->dtype == MOE_BF16 ? 0 : 1, st) == cudaSuccess ? MOE_OK
+                                                                                  : MOE_ERR_CUDA;
+}
