@@ -126,6 +126,24 @@ def algorithmic_bytes(shape, dbg, B):
             "rows": sum(len(u) for u in union.values())}
 
 
+def traffic_of(key):
+    """DRAM bytes (read + write) of one launch from the committed ncu capture of that kernel,
+    or None when there is none or the kernel's sources changed since it was taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        ent = json.load(f).get(key)
+    if not ent:
+        return None
+    h = hashlib.sha256()
+    for name in ent["source_files"]:
+        with open(os.path.join(ROOT, "sparse_expert_ffn_logits_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return ent["bytes"] if h.hexdigest()[:16] == ent["source_sha"] else None
+
+
 def run_cuda(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -240,12 +258,7 @@ def run_cuda(args, rank, world, local_rank):
     peak, peak_kind = peaks()
     achieved = abytes[dom] / (stage_avg[dom] / 1e3) / 1e9
     layer_bytes = sum(abytes[n] for n in ("router", "gate", "updown"))
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tpath):
-        with open(tpath) as f:
-            tr = json.load(f).get(f"{args.workload}:B{B}:s{s}:{dom}")
-        traffic = tr
+    traffic = traffic_of(f"{args.workload}:B{B}:s{s}:{dom}")
     roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
                 "peak_source": f"hbm copy, {peak_kind}", "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,
