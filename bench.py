@@ -356,7 +356,7 @@ def cpu_baseline(shape, B, rule, seconds):
                synth.host_tensor(shape, "sh_down", j)) for j in range(shape.n_shared)]
     cache = {}
     done_tok, spent, nb = 0, 0.0, 0
-    while spent < seconds and nb < 64:
+    while spent < seconds and nb < 4096:
         x = synth.host_tokens(shape, B, synth.token_seed(shape, nb))
         _, idx, _ = rl.route(x)
         need = sorted(set(int(e) for e in idx.ravel()))
