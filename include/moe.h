@@ -170,6 +170,16 @@ moe_status moe_read_trace(moe_handle* h, unsigned long long* host, size_t n);
  * MOE_OK with *device_code = 0. */
 moe_status moe_get_error(moe_handle* h, int* device_code);
 
+/* Path choice per expert.  An expert (routed or shared) that receives at least min_tokens tokens
+ * in a call is computed by the dense masked path on the tensor cores (gate GEMM, the same
+ * selection, up GEMM times the 0/1 mask and SiLU(g), down GEMM), the others by the sparse
+ * kernels; both compute the same function ("Uncovering Intra-expert Activation Sparsity ...",
+ * technical summary, Methodology: sparse or dense kernels chosen by batch size).  min_tokens = 0
+ * turns the dense path off; bf16 layers only (fp32 layers always take the sparse kernels).
+ * The default comes from the crossover measured on B200.  INVALID_ARG for a NULL handle or a
+ * negative count.  Takes effect from the next moe_forward. */
+moe_status moe_set_dense_min_tokens(moe_handle* h, int min_tokens);
+
 /* Frees the workspace and the handle (synchronises the device first).  NULL is a no-op. */
 moe_status moe_destroy(moe_handle* h);
 

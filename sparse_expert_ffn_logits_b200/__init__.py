@@ -51,7 +51,8 @@ _LIB = None
 # C entry points declared in include/moe.h
 EXPORTS = ("moe_create", "moe_packed_bytes", "moe_pack_experts", "moe_forward",
            "moe_forward_host", "moe_debug_lists", "moe_profile_stages", "moe_read_trace",
-           "moe_get_error", "moe_destroy", "moe_route_noalloc", "moe_status_string")
+           "moe_get_error", "moe_set_dense_min_tokens", "moe_destroy", "moe_route_noalloc",
+           "moe_status_string")
 MOE_STAGE_EVENTS = 6
 STAGES = ("router", "gate", "select", "updown", "finalize")
 
@@ -78,6 +79,7 @@ def _lib():
         lib.moe_read_trace.argtypes = [P, P, ctypes.c_size_t]
         lib.moe_get_error.argtypes = [P, ctypes.POINTER(I)]
         lib.moe_destroy.argtypes = [P]
+        lib.moe_set_dense_min_tokens.argtypes = [P, I]
         lib.moe_route_noalloc.argtypes = [ctypes.POINTER(MoEConfig), P, I, P, P, P, P]
         lib.moe_status_string.argtypes = [I]
         lib.moe_status_string.restype = ctypes.c_char_p
@@ -203,6 +205,12 @@ def moe_get_error(h):
     if rc not in (MOE_OK, MOE_ERR_DEVICE):
         raise MoEError(rc, "moe_get_error")
     return rc, code.value
+
+
+def moe_set_dense_min_tokens(h, min_tokens):
+    """Experts with at least min_tokens tokens take the tensor-core path (0: never)."""
+    _check(_lib().moe_set_dense_min_tokens(ctypes.c_void_p(h) if h else None, int(min_tokens)),
+           "moe_set_dense_min_tokens")
 
 
 def moe_destroy(h):

@@ -96,6 +96,11 @@ struct FwdParams {
   const void* zero_row;  // H zero elements (source of the copies of absent tokens)
   unsigned long long* trace;  // per-CTA phase timestamps (nullptr: tracing off)
   unsigned* claim;            // [2] work-item counters of the gate and up/down kernels
+  // dense masked fallback: a slot with T >= dense_min tokens is computed by the tcgen05 GEMMs
+  int dense_min;              // INT_MAX: never
+  int imax_pad;               // Imax rounded up to 128 (row length of hbuf)
+  __nv_bfloat16* xp;          // [Pmax][H] x rows of the pairs of dense slots
+  __nv_bfloat16* hbuf;        // [Pmax][imax_pad] mask * SiLU(g) * u of dense slots, bf16
 };
 
 // Phase timestamps for tracing: kernel k, CTA b, point i (i < kTracePoints).
@@ -149,9 +154,18 @@ __device__ __forceinline__ int ld_cg(const int* p) { return __ldcg(p); }
 __device__ __forceinline__ unsigned ld_cg(const unsigned* p) { return __ldcg(p); }
 __device__ __forceinline__ float ld_cg(const float* p) { return __ldcg(p); }
 
+// bitwise OR into global memory, no value returned (an atomicOr whose result is unused may
+// still wait for it)
+__device__ __forceinline__ void red_or(uint32_t* p, uint32_t v) {
+  asm volatile("red.global.or.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // fp32 vector reductions into global memory (sm_90+); v4 needs a 16-byte aligned address
 __device__ __forceinline__ void red_add_v2(float* p, float a, float b) {
   asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(a), "f"(b) : "memory");
+}
+__device__ __forceinline__ void red_add_f32(float* p, float a) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(a) : "memory");
 }
 __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),

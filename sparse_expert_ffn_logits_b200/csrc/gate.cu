@@ -61,6 +61,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, 
   uint64_t* mempty = mfull + kMetaRing;
   uint64_t* xfull = mempty + kMetaRing;
   uint64_t* xempty = xfull + 2;
+  uint64_t* mrows = xempty + 2;  // the record's row pointer is written (all the copier needs)
   float(*red)[kWarps][4][32] = reinterpret_cast<float(*)[kWarps][4][32]>(smem + kBarBytes);
   unsigned char* xbuf = smem + kBarBytes + kRedBytes;
   unsigned char* ring = xbuf + rc.nxb * rc.xs_bytes;
@@ -74,6 +75,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, 
     for (int i = 0; i < kMetaRing; ++i) {
       mbar_init(&mfull[i], 1);
       mbar_init(&mempty[i], kWarps + 1);
+      mbar_init(&mrows[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&xfull[i], 1);
@@ -87,17 +89,21 @@ __global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, 
   pdl_trigger();
   pdl_wait();
   trace_point(p.trace, 1, 1);
+  // the slot count and every slot entry that can exist (E + S) in one round trip; entries at
+  // n_slots and beyond are stale and never searched
   const int n_slots = ld_cg(&p.meta[kMetaSlots]);
   const int n_items = ld_cg(&p.meta[kMetaGateItems]);
-  load_slot_table(p, n_slots, s_tab);
+  load_slot_table(p, min(p.E + p.S, kMaxSlots), s_tab);
   __syncthreads();
   const int H = p.H;
   volatile int* abort = &s_abort;
 
   if (warp == kMetaWarp) {
     // ---------------- meta: claims items (its own contiguous share first, then a few at a time
-    // from the work counter, so that fast CTAs take more of the tail), publishes their records one item ahead of the copier and the consumers,
-    // and (generic variant) fills the token tiles.  A record with end = 1 closes the stream.
+    // from the work counter, so that fast CTAs take more of the tail) and publishes their
+    // records: the row pointer for the copier (mrows), then the tokens for the consumers
+    // (mfull); it also fills the token tiles of the generic variant.  A record with end = 1
+    // closes the stream.
     int xuse[2] = {0, 0};
     // a contiguous share of 7/8 of the items (token tiles stay together), then the rest from
     // the counter in small chunks
@@ -137,6 +143,18 @@ __global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, 
       const int I = kind ? p.Ish : p.I;
       const int local = cur - sl.w, tt = local / (I / kTileRows), rg = local % (I / kTileRows);
       const int nt = min(kTileTok, T - tt * kTileTok);
+      if (lane == 0) {  // the copier's part first: it needs no token
+        const __nv_bfloat16* base =
+            kind == 0 ? static_cast<const __nv_bfloat16*>(p.gate_r) + (size_t)ex * p.I * H
+                      : static_cast<const __nv_bfloat16*>(p.gate_s) + (size_t)ex * p.Ish * H;
+        s_meta[m].rows = base + (size_t)rg * kTileRows * H;
+        s_meta[m].q0 = q0 + tt * kTileTok;
+        s_meta[m].nt = nt;
+        s_meta[m].n0 = rg * kTileRows;
+        s_meta[m].key = cur_key;
+        s_meta[m].end = 0;
+        mbar_arrive(&mrows[m]);
+      }
       int xpar = 0;
       if (cur_key != key) {
         key = cur_key;
@@ -161,18 +179,9 @@ __global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, 
       }
       if (lane < kTileTok) s_meta[m].tok[lane] = tok_l;
       if (lane == 0) {
-        const __nv_bfloat16* base =
-            kind == 0 ? static_cast<const __nv_bfloat16*>(p.gate_r) + (size_t)ex * p.I * H
-                      : static_cast<const __nv_bfloat16*>(p.gate_s) + (size_t)ex * p.Ish * H;
-        s_meta[m].rows = base + (size_t)rg * kTileRows * H;
-        s_meta[m].q0 = q0 + tt * kTileTok;
-        s_meta[m].nt = nt;
-        s_meta[m].n0 = rg * kTileRows;
-        s_meta[m].key = key;
         s_meta[m].xb = xb;
         s_meta[m].xpar = xpar;
         s_meta[m].xlast = nxt_key != key;
-        s_meta[m].end = 0;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&mfull[m]);
@@ -184,6 +193,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, 
       mbar_wait(&mempty[m], ((mi / kMetaRing) & 1) ^ 1, abort, p.err);
       if (lane == 0) {
         s_meta[m].end = 1;
+        mbar_arrive(&mrows[m]);
         mbar_arrive(&mfull[m]);
       }
     }
@@ -199,7 +209,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, 
     int it = 0;
     for (int mi = 0; !*abort; ++mi) {
       const int m = mi % kMetaRing;
-      if (!mbar_wait(&mfull[m], (mi / kMetaRing) & 1, abort, p.err)) break;
+      if (!mbar_wait(&mrows[m], (mi / kMetaRing) & 1, abort, p.err)) break;
       if (s_meta[m].end) break;
       const __nv_bfloat16* row = s_meta[m].rows + (size_t)(lane & 15) * H;
       __syncwarp();

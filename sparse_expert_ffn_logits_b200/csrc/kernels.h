@@ -27,6 +27,10 @@ cudaError_t launch_gate(const FwdParams& p, int dtype, const LaunchShape& ls, cu
 cudaError_t launch_select(const FwdParams& p, const LaunchShape& ls, cudaStream_t st, bool pdl);
 cudaError_t launch_updown(const FwdParams& p, int dtype, const LaunchShape& ls, cudaStream_t st,
                           bool pdl);
+// dense masked fallback (dense.cu): stage 0 = gather + gate GEMM, stage 1 = up + down GEMMs
+cudaError_t launch_dense(const FwdParams& p, const LaunchShape& ls, int stage, cudaStream_t st,
+                         bool pdl);
+cudaError_t configure_dense(int budget);
 cudaError_t launch_finalize(const FwdParams& p, int dtype, const LaunchShape& ls, cudaStream_t st,
                             bool pdl);
 

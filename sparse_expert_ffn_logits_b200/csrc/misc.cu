@@ -121,6 +121,10 @@ cudaError_t configure_kernels(int dtype, int imax, int max_E, int max_B, int H, 
   if (e != cudaSuccess) return e;
   e = configure_updown(dtype, H, budget, ls);
   if (e != cudaSuccess) return e;
+  if (dtype == 0) {
+    e = configure_dense(budget);
+    if (e != cudaSuccess) return e;
+  }
   return cudaGetLastError();
 }
 

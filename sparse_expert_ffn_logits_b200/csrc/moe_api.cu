@@ -16,6 +16,8 @@
 
 #include <new>
 
+#include <climits>
+
 #include "../../include/moe.h"
 #include "kernels.h"
 
@@ -39,10 +41,15 @@ struct moe_handle {
   int last_tokens;
   cudaEvent_t stage_events[MOE_STAGE_EVENTS];
   bool timing;
+  int dense_min;  // tokens of a slot from which the tensor-core path computes it (0: never)
   unsigned long long* trace_buf;  // device, kTraceKernels * kTraceCtas * kTracePoints stamps
 };
 
 namespace {
+
+// Tokens per expert from which a slot goes to the tensor-core path by default (measured on
+// B200: see the design notes' crossover table); moe_set_dense_min_tokens overrides it.
+constexpr int kDefaultDenseMin = 48;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -124,6 +131,11 @@ size_t carve(moe_handle* h, char* base) {
   p.trace = nullptr;
   h->x_stage = cv.take<char>(Bm * c.hidden * h->elt);
   h->out_stage = cv.take<char>(Bm * c.hidden * h->elt);
+  // dense fallback buffers (bf16 layers only)
+  p.imax_pad = (int)((Im + 127) / 128 * 128);
+  const bool dense_ok = c.dtype == MOE_BF16;
+  p.xp = dense_ok ? cv.take<__nv_bfloat16>(Pm * c.hidden) : nullptr;
+  p.hbuf = dense_ok ? cv.take<__nv_bfloat16>(Pm * (size_t)p.imax_pad) : nullptr;
   // zero-at-rest region: tickets, union bitmasks, output accumulator
   char* zb = cv.take<char>(0);
   p.tile_ticket = cv.take<unsigned>((Bm + moe::kTileTok - 1) / moe::kTileTok);
@@ -185,14 +197,21 @@ moe_status forward_impl(moe_handle* h, const void* x, int n_tokens, const void* 
   static const bool no_pdl = getenv("MOE_NO_PDL") != nullptr && getenv("MOE_NO_PDL")[0] == '1';
   const bool tm = h->timing, pdl = !tm && !no_pdl;
   p.trace = tm ? h->trace_buf : nullptr;
+  // dense fallback: slots with at least dense_min tokens (bf16 only; no slot has more than
+  // n_tokens tokens, so below that nothing is launched for it).  The router already needs it:
+  // it gives dense slots no sparse gate items.
+  p.dense_min = (dt == 0 && h->dense_min > 0) ? h->dense_min : INT_MAX;
+  const bool dense = p.dense_min <= n_tokens;
   cudaEvent_t* ev = h->stage_events;
   cudaError_t e = tm ? cudaEventRecord(ev[0], st) : cudaSuccess;
   if (e == cudaSuccess) e = moe::launch_router(p, dt, st);
   if (e == cudaSuccess && tm) e = cudaEventRecord(ev[1], st);
   if (e == cudaSuccess) e = moe::launch_gate(p, dt, h->ls, st, pdl);
+  if (e == cudaSuccess && dense) e = moe::launch_dense(p, h->ls, 0, st, pdl);
   if (e == cudaSuccess && tm) e = cudaEventRecord(ev[2], st);
   if (e == cudaSuccess) e = moe::launch_select(p, h->ls, st, pdl);
   if (e == cudaSuccess && tm) e = cudaEventRecord(ev[3], st);
+  if (e == cudaSuccess && dense) e = moe::launch_dense(p, h->ls, 1, st, pdl);
   if (e == cudaSuccess) e = moe::launch_updown(p, dt, h->ls, st, pdl);
   if (e == cudaSuccess && tm) e = cudaEventRecord(ev[4], st);
   if (e == cudaSuccess) e = moe::launch_finalize(p, dt, h->ls, st, pdl);
@@ -258,6 +277,7 @@ moe_status moe_create(const moe_config* cfg, moe_handle** out) {
     delete h;
     return MOE_ERR_OOM;
   }
+  h->dense_min = kDefaultDenseMin;
   carve(h, static_cast<char*>(h->ws));
   if (cudaMemset(h->ws, 0, h->ws_bytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
     cudaFree(h->ws);
@@ -397,6 +417,12 @@ moe_status moe_get_error(moe_handle* h, int* device_code) {
   *device_code = v;
   if (cudaMemset(h->base.err, 0, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_ERR_DEVICE;
+}
+
+moe_status moe_set_dense_min_tokens(moe_handle* h, int min_tokens) {
+  if (!h || min_tokens < 0) return MOE_ERR_INVALID_ARG;
+  h->dense_min = min_tokens;
+  return MOE_OK;
 }
 
 moe_status moe_destroy(moe_handle* h) {

@@ -17,6 +17,7 @@
 // later call only clears the zero-at-start words and launches.  Calls that overlap in time on one
 // device, from two streams or two threads, share the scratch area and race: the caller
 // serialises them.
+#include <climits>
 #include <mutex>
 
 #include "../../include/moe.h"
@@ -131,6 +132,7 @@ extern "C" moe_status moe_route_noalloc(const moe_config* cfg, const void* x, in
   p.Bmax = B;
   p.hsplit = hsplit;
   p.route = (int)cfg->route;
+  p.dense_min = INT_MAX;  // only the grouping's item counts read it; no later kernel runs
   p.x = x;
   p.router = router;
   p.logits = reinterpret_cast<float*>(base + o_logits);

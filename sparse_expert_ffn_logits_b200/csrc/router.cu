@@ -158,8 +158,11 @@ __device__ void group_pairs(const FwdParams& p, uint32_t* dyn, unsigned long lon
   unsigned long long mine = 0ull;
   for (int e = e0; e < e1; ++e) {
     const unsigned long long c = (unsigned)cnt[e];
+    // a dense slot (c >= dense_min) has no sparse gate items: the tensor-core path covers it
     const unsigned long long items =
-        c ? (unsigned long long)(p.I / kTileRows) * ((c + kTileTok - 1) / kTileTok) : 0ull;
+        c && (int)c < p.dense_min
+            ? (unsigned long long)(p.I / kTileRows) * ((c + kTileTok - 1) / kTileTok)
+            : 0ull;
     mine += c | ((c ? 1ull : 0ull) << 20) | (items << 32);
   }
   unsigned long long tot;
@@ -168,14 +171,16 @@ __device__ void group_pairs(const FwdParams& p, uint32_t* dyn, unsigned long lon
     pre[e] = run;
     const unsigned long long c = (unsigned)cnt[e];
     run += c | ((c ? 1ull : 0ull) << 20) |
-           ((c ? (unsigned long long)(p.I / kTileRows) * ((c + kTileTok - 1) / kTileTok) : 0ull)
+           ((c && (int)c < p.dense_min
+                 ? (unsigned long long)(p.I / kTileRows) * ((c + kTileTok - 1) / kTileTok)
+                 : 0ull)
             << 32);
   }
   __syncthreads();
   const int n_touched = (int)((tot >> 20) & 0xFFF);
   const int routed_items = (int)(tot >> 32);
   const int n_slots = n_touched + S;
-  const int sh_items = (p.Ish / kTileRows) * ((B + kTileTok - 1) / kTileTok);
+  const int sh_items = B < p.dense_min ? (p.Ish / kTileRows) * ((B + kTileTok - 1) / kTileTok) : 0;
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     if (cnt[e] > 0) {
       const unsigned long long pr = pre[e];

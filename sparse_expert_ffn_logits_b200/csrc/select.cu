@@ -3,12 +3,13 @@
 // Inside a pair the lowest-scoring neuron activations are dropped ("Uncovering Intra-expert
 // Activation Sparsity ...", technical summary, Methodology: activation masking).  The score of
 // neuron n is |SiLU(g_n)|, an fp32 value whose bit pattern (sign cleared) orders like the value.
-//   top-K mode: an MSB-first radix select (eight 4-bit digits) finds the K-th largest key tau
-//     and how many keys equal to tau are kept; the kept set is every key > tau plus the
-//     lowest-indexed keys == tau.  No sort.
+//   top-K mode: an MSB-first radix select (4-bit digits) finds the K-th largest key tau and
+//     how many keys equal to tau are kept; the kept set is every key > tau plus the
+//     lowest-indexed keys == tau.  No sort.  Once at most 32 keys share the decided prefix,
+//     one warp ranks those directly.
 //   threshold mode: one pass, keep key > t (the page's single-pass threshold mask).
 // One CTA per pair: its keys sit in shared memory; each radix pass counts digits in registers
-// (packed 16-bit bins) and merges them with warp reductions, with no atomics.  The kept set is
+// (packed 16-bit bins), merges them with warp reductions and one barrier.  The kept set is
 // written as an ascending index list + count (for export), as a bitmask row, and
 // OR-ed into the expert's union bitmask.  The last pair of an expert to finish (atomic ticket,
 // no waiting) compacts the union into an ascending row list for the up/down kernel and clears
@@ -23,48 +24,57 @@ constexpr int kSelWarps = kSelThreads / 32;
 
 __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
   extern __shared__ uint32_t sm[];
-  __shared__ int hist[2048];
+  __shared__ int hist[2 * kSelWarps * 8];
   __shared__ int scratch[33];
-  __shared__ int wtot[kSelWarps];
-  __shared__ int s_digit, s_above, s_last;
+  __shared__ uint32_t cbuf[32];
+  __shared__ int s_ncand, s_need, s_last;
+  __shared__ uint32_t s_tau;
   pdl_trigger();
   trace_point(p.trace, 2, 0);
   pdl_wait();
   trace_point(p.trace, 2, 1);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int Imax = p.Imax, Wmax = p.Imax / 32;
-  uint32_t* key = sm;                                                 // [Imax]
-  unsigned char* keep = reinterpret_cast<unsigned char*>(sm + Imax);  // [Imax]
+  uint32_t* key = sm;  // [Imax]
   const int n_pairs = ld_cg(&p.meta[kMetaPairs]);
   bool nan_seen = false;
   for (int q = blockIdx.x; q < n_pairs; q += gridDim.x) {
-    const int j = __ldcg(&p.pair_slot[q]);
-    const Slot s = load_slot(&p.slots[j]);
-    const int I = s.I, kind = s.kind;
-    {
-      const float4* a4 = reinterpret_cast<const float4*>(p.act + (size_t)q * Imax);
-      for (int v0 = threadIdx.x; v0 < I / 4; v0 += 4 * kSelThreads) {
-        float4 f[4];  // four 16-byte loads in flight per thread
+    // The first activations are requested before the pair's slot is known (the row is Imax
+    // long whatever the expert's I): one round trip instead of three dependent ones.
+    const float4* a4 = reinterpret_cast<const float4*>(p.act + (size_t)q * Imax);
+    float4 f[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          f[u] = v0 + u * kSelThreads < I / 4 ? __ldcg(a4 + v0 + u * kSelThreads)
-                                              : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int u = 0; u < 4; ++u) {
+      const int v = threadIdx.x + u * kSelThreads;
+      f[u] = v < Imax / 4 ? __ldcg(a4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    // routed pairs come first (B * k of them), then the shared experts' pairs
+    const int kind = q >= p.B * p.k ? 1 : 0;
+    const int I = kind ? p.Ish : p.I;
+    const int j = __ldcg(&p.pair_slot[q]);  // needed only for the union, after the selection
+    if (threadIdx.x == 0) s_ncand = 0;
+    for (int v0 = threadIdx.x;; v0 += 4 * kSelThreads) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int v = v0 + u * kSelThreads;
-          if (v < I / 4) {
-            const float fv[4] = {f[u].x, f[u].y, f[u].z, f[u].w};
+      for (int u = 0; u < 4; ++u) {
+        const int v = v0 + u * kSelThreads;
+        if (v < I / 4) {
+          const float fv[4] = {f[u].x, f[u].y, f[u].z, f[u].w};
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              uint32_t k4 = __float_as_uint(fabsf(fv[c]));
-              if (isnan(fv[c])) {
-                nan_seen = true;
-                k4 = 0;
-              }
-              key[v * 4 + c] = k4;
+          for (int c = 0; c < 4; ++c) {
+            uint32_t k4 = __float_as_uint(fabsf(fv[c]));
+            if (isnan(fv[c])) {
+              nan_seen = true;
+              k4 = 0;
             }
+            key[v * 4 + c] = k4;
           }
         }
+      }
+      if (v0 + 4 * kSelThreads >= I / 4) break;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {  // the next four 16-byte loads per thread
+        const int v = v0 + 4 * kSelThreads + u * kSelThreads;
+        f[u] = v < I / 4 ? __ldcg(a4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
     __syncthreads();
@@ -76,15 +86,17 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
     uint32_t tau = 0;
     int need = 0;
     if (radix) {
-      // eight 4-bit digits, most significant first.  Each thread counts its keys per digit in
-      // packed 16-bit fields (bins 2i, 2i+1 in c[i]), a warp sum merges them, and warp 0 reads
-      // the eight warps' sums to pick the digit: no atomics, two barriers per digit.
+      // MSB-first radix select of the K-th largest key, 4-bit digits.  Each thread counts its
+      // keys per digit in packed 16-bit fields, a warp sum merges them, and after one barrier
+      // every warp reads the eight warps' sums and finds the digit itself (the histogram is
+      // double-buffered, so the next pass can write while a slow warp still reads).  Once at
+      // most 32 keys share the prefix, one warp ranks them directly.
       uint32_t prefix = 0, pmask = 0;
-      int krem = K;
+      int krem = K, cand = I, shift = 28, pass = 0;
 #pragma unroll 1
-      for (int shift = 28; shift >= 0; shift -= 4) {
+      for (; shift >= 0 && cand > 32; shift -= 4, ++pass) {
         uint32_t c[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        for (int n = threadIdx.x; n < I; n += blockDim.x) {
+        for (int n = threadIdx.x; n < I; n += kSelThreads) {
           const uint32_t u = key[n];
           if ((u & pmask) == prefix) {
             const uint32_t d = (u >> shift) & 15u;
@@ -95,111 +107,151 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) c[i] = __reduce_add_sync(0xffffffffu, c[i]);
+        int* hb = hist + (pass & 1) * (kSelWarps * 8);
         if (lane == 0) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) hist[warp * 8 + i] = (int)c[i];
+          for (int i = 0; i < 8; ++i) hb[warp * 8 + i] = (int)c[i];
+        }
+        __syncthreads();
+        // lane l < 16 holds digit 15 - l; a scan over the lanes finds the digit of the K-th key
+        int cnt = 0;
+        if (lane < 16) {
+          const int d = 15 - lane;
+#pragma unroll
+          for (int w = 0; w < kSelWarps; ++w)
+            cnt += (int)(((uint32_t)hb[w * 8 + (d >> 1)] >> ((d & 1) * 16)) & 0xFFFFu);
+        }
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const int above = incl - cnt;
+        const unsigned hit = __ballot_sync(0xffffffffu, lane < 16 && above < krem && incl >= krem);
+        const int src = __ffs(hit) - 1;
+        krem -= __shfl_sync(0xffffffffu, above, src);
+        cand = __shfl_sync(0xffffffffu, cnt, src);
+        prefix |= (uint32_t)(15 - src) << shift;
+        pmask |= 15u << shift;
+      }
+      if (shift < 0) {
+        tau = prefix;  // every bit decided: the krem largest keys equal to prefix are kept
+        need = krem;
+      } else {
+        // at most 32 keys carry the prefix: gather them (any order) and rank them in warp 0
+        for (int n = threadIdx.x; n < I; n += kSelThreads) {
+          const uint32_t u = key[n];
+          if ((u & pmask) == prefix) {
+            const int slot = atomicAdd(&s_ncand, 1);  // < cand <= 32 by construction
+            if (slot < 32) cbuf[slot] = u;
+          }
         }
         __syncthreads();
         if (warp == 0) {
-          // lane l < 16 holds digit 15 - l; a suffix scan over the lanes finds the digit
-          int cnt = 0;
-          if (lane < 16) {
-            const int d = 15 - lane;
-#pragma unroll
-            for (int w = 0; w < kSelWarps; ++w)
-              cnt += (int)(((uint32_t)hist[w * 8 + (d >> 1)] >> ((d & 1) * 16)) & 0xFFFFu);
+          const bool valid = lane < cand;
+          const uint32_t mine = valid ? cbuf[lane] : 0u;
+          int gt = 0, ge = 0;
+          for (int j = 0; j < cand; ++j) {
+            const uint32_t o = __shfl_sync(0xffffffffu, mine, j);
+            gt += o > mine;
+            ge += o >= mine;
           }
-          int incl = cnt;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
-          }
-          const int above = incl - cnt;
-          const unsigned hit = __ballot_sync(0xffffffffu, lane < 16 && above < krem && incl >= krem);
+          const unsigned hit = __ballot_sync(0xffffffffu, valid && gt < krem && ge >= krem);
           const int src = __ffs(hit) - 1;
           if (lane == src) {
-            s_digit = 15 - lane;
-            s_above = above;
+            s_tau = mine;
+            s_need = krem - gt;
           }
         }
         __syncthreads();
-        krem -= s_above;
-        prefix |= (uint32_t)s_digit << shift;
-        pmask |= 15u << shift;
+        tau = s_tau;
+        need = s_need;
       }
-      tau = prefix;
-      need = krem;
     }
     if (q == (int)blockIdx.x) trace_point(p.trace, 2, 3);
-    // warp-contiguous segments of the neuron range, walked 32 at a time (ordered ballots)
-    const int seg = ((I + 32 * kSelWarps - 1) / (32 * kSelWarps)) * 32;
-    const int sb = warp * seg, se = min(I, sb + seg);
-    int tie_base = 0;
-    if (radix) {
-      int ties = 0;
-      for (int n0 = sb; n0 < se; n0 += 32) {
-        const int n = n0 + lane;
-        ties += __popc(__ballot_sync(0xffffffffu, n < se && key[n] == tau));
-      }
-      if (lane == 0) wtot[warp] = ties;
-      __syncthreads();
-      for (int w = 0; w < warp; ++w) tie_base += wtot[w];
-      __syncthreads();
-    }
-    int kept = 0;
-    {
-      int run = tie_base;
-      for (int n0 = sb; n0 < se; n0 += 32) {
-        const int n = n0 + lane;
-        const uint32_t u = n < se ? key[n] : 0u;
-        bool k_n;
-        if (mode == 1) {
-          k_n = __uint_as_float(u) > thr;
-        } else if (K >= I) {
-          k_n = true;
-        } else if (K == 0) {
-          k_n = false;
-        } else {
-          const bool eq = n < se && u == tau;
-          const unsigned be = __ballot_sync(0xffffffffu, eq);
-          k_n = u > tau || (eq && run + __popc(be & lanemask_lt()) < need);
-          run += __popc(be);
-        }
-        k_n = k_n && n < se;
-        if (n < se) keep[n] = k_n ? 1 : 0;
-        kept += __popc(__ballot_sync(0xffffffffu, k_n));
+    // Kept set, chunk-parallel.  Chunk c = neurons 32c .. 32c + 31 (one ballot each).
+    //   A: every warp takes chunks warp, warp + 8, ...: masks of keys above the cut and equal to
+    //      it (ties exist only in top-K mode).
+    //   B: warp 0 scans the chunks in order: ties are kept lowest index first, so chunk c keeps
+    //      the first min(eq_c, need - ties before c) of its ties; it writes each chunk's kept
+    //      mask and its first list position.
+    //   C: every warp writes its chunks' list entries, mask words and union bits.
+    const int nch = I / 32;
+    uint32_t* s_km = key + Imax;           // [Imax / 32] above-cut mask, then the kept mask
+    uint32_t* s_em = s_km + Imax / 32;     // [Imax / 32] tie mask
+    int* s_pos = reinterpret_cast<int*>(s_em + Imax / 32);  // [Imax / 32] first list position
+    for (int c = warp; c < nch; c += kSelWarps) {
+      const uint32_t u = key[32 * c + lane];
+      bool above;
+      if (mode == 1) above = __uint_as_float(u) > thr;
+      else if (K >= I) above = true;
+      else if (K == 0) above = false;
+      else above = u > tau;
+      const unsigned gm = __ballot_sync(0xffffffffu, above);
+      const unsigned em = __ballot_sync(0xffffffffu, radix && u == tau);
+      if (lane == 0) {
+        s_km[c] = gm;
+        s_em[c] = em;
       }
     }
-    if (lane == 0) wtot[warp] = kept;
     __syncthreads();
-    int pos = 0, total = 0;
-    for (int w = 0; w < kSelWarps; ++w) {
-      if (w < warp) pos += wtot[w];
-      total += wtot[w];
+    if (warp == 0) {
+      // lane l owns the contiguous chunk block [l * cpl, (l + 1) * cpl)
+      const int cpl = (nch + 31) / 32;
+      const int c0 = min(nch, lane * cpl), c1 = min(nch, c0 + cpl);
+      int ties = 0;
+      for (int c = c0; c < c1; ++c) ties += __popc(s_em[c]);
+      int tincl = ties;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, tincl, o);
+        if (lane >= o) tincl += y;
+      }
+      int tb = tincl - ties;  // ties before this lane's block
+      int kept = 0;
+      for (int c = c0; c < c1; ++c) {
+        uint32_t em = s_em[c];
+        const int ne = __popc(em);
+        const int take = max(0, min(ne, need - tb));
+        for (int d = ne - take; d > 0; --d) em ^= 1u << (31 - __clz(em));  // drop the highest
+        const uint32_t km = s_km[c] | em;
+        s_km[c] = km;
+        tb += ne;
+        kept += __popc(km);
+      }
+      int kincl = kept;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, kincl, o);
+        if (lane >= o) kincl += y;
+      }
+      int kb = kincl - kept;
+      for (int c = c0; c < c1; ++c) {
+        s_pos[c] = kb;
+        kb += __popc(s_km[c]);
+      }
+      if (lane == 31) p.cnt[q] = kincl;
     }
+    __syncthreads();
     int* list = p.lists + (size_t)q * Imax;
     uint32_t* mrow = p.maskbits + (size_t)q * Wmax;
     uint32_t* urow = p.ubits + (size_t)j * Wmax;
-    for (int n0 = sb; n0 < se; n0 += 32) {
-      const int n = n0 + lane;
-      const bool k_n = n < se && keep[n];
-      const unsigned b = __ballot_sync(0xffffffffu, k_n);
-      if (k_n) list[pos + __popc(b & lanemask_lt())] = n;
-      pos += __popc(b);
+    for (int c = warp; c < nch; c += kSelWarps) {
+      const uint32_t km = s_km[c];
+      if ((km >> lane) & 1u) list[s_pos[c] + __popc(km & lanemask_lt())] = 32 * c + lane;
       if (lane == 0) {
-        mrow[n0 >> 5] = b;
-        if (b) atomicOr(&urow[n0 >> 5], b);
+        mrow[c] = km;
+        if (km) red_or(&urow[c], km);
       }
     }
-    if (threadIdx.x == 0) p.cnt[q] = total;
     if (q == (int)blockIdx.x) trace_point(p.trace, 2, 4);
     __threadfence();
     __syncthreads();
     if (q == (int)blockIdx.x) trace_point(p.trace, 2, 5);
     if (threadIdx.x == 0) {
       const unsigned ticket = atomicAdd(&p.slot_ticket[j], 1u);
-      s_last = ticket == (unsigned)s.T - 1u;
+      s_last = ticket == (unsigned)__ldcg(&p.slots[j].T) - 1u;
     }
     __syncthreads();
     if (q == (int)blockIdx.x) trace_point(p.trace, 2, 6);
@@ -239,7 +291,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
 
 }  // namespace
 
-size_t select_smem_bytes(int imax) { return (size_t)imax * 5 + 16; }
+// keys [Imax] | kept masks, tie masks, list positions [Imax / 32] each
+size_t select_smem_bytes(int imax) { return (size_t)imax * 4 + (size_t)(imax / 32) * 12 + 16; }
 
 cudaError_t launch_select(const FwdParams& p, const LaunchShape& ls, cudaStream_t st, bool pdl) {
   const int pairs = p.B * (p.k + p.S);

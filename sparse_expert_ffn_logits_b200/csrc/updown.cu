@@ -109,6 +109,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
   uint64_t* xfull = mempty + kMetaRing;
   uint64_t* xempty = xfull + 2;
   uint64_t* mhead = xempty + 2;  // the lead warp has written the record's item
+  uint64_t* mrows = mhead + kMetaRing;  // the record's rows are written (all the copier needs)
   float(*red)[kWarps][4][32] = reinterpret_cast<float(*)[kWarps][4][32]>(smem + kBarBytes);
   unsigned char* xbuf = smem + kBarBytes + kRedBytes;
   unsigned char* ring = xbuf + rc.nxb * rc.xs_bytes;
@@ -123,6 +124,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
       mbar_init(&mfull[i], 2);  // lead meta warp + the coefficient warp of that record
       mbar_init(&mempty[i], kWarps + 1);
       mbar_init(&mhead[i], 1);
+      mbar_init(&mrows[i], 2);  // lead meta warp + the coefficient warp of that record
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&xfull[i], 1);
@@ -138,13 +140,17 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
   trace_point(p.trace, 3, 1);
   const int n_slots = ld_cg(&p.meta[kMetaSlots]);
   {
-    // items per slot = ceil(union rows / 16) * token tiles; exclusive prefix into s_tab[].w
-    const int per = (n_slots + blockDim.x - 1) / blockDim.x;
-    const int b0 = min(n_slots, (int)threadIdx.x * per), b1 = min(n_slots, b0 + per);
+    // items per slot = ceil(union rows / 16) * token tiles; exclusive prefix into s_tab[].w.
+    // Every slot entry that can exist (E + S) is read together with the slot count (one round
+    // trip); entries at n_slots and beyond count as empty.
+    const int n_max = min(p.E + p.S, kMaxSlots);
+    const int per = (n_max + blockDim.x - 1) / blockDim.x;
+    const int b0 = min(n_max, (int)threadIdx.x * per), b1 = min(n_max, b0 + per);
     int c = 0;
     for (int j = b0; j < b1; ++j) {
       const Slot sl = load_slot(&p.slots[j]);
-      const int rows = __ldcg(&p.ucnt[j]);
+      const int rows_any = __ldcg(&p.ucnt[j]);  // issued before n_slots is known
+      const int rows = j < n_slots && sl.T < p.dense_min ? rows_any : 0;  // dense: not here
       s_ucnt[j] = rows;
       const int v = ((rows + kTileRows - 1) / kTileRows) * ((sl.T + kTileTok - 1) / kTileTok);
       s_tab[j] = make_int4(sl.expert | (sl.kind << 16), sl.T, sl.q0, v);
@@ -249,6 +255,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
         s_meta[m].rg = cp.rg;
         s_meta[m].end = 0;
         mbar_arrive(&mhead[m]);
+        mbar_arrive(&mrows[m]);
         mbar_arrive(&mfull[m]);
       }
       __syncwarp();
@@ -261,6 +268,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
       if (lane == 0) {
         s_meta[m].end = 1;
         mbar_arrive(&mhead[m]);
+        mbar_arrive(&mrows[m]);
         mbar_arrive(&mfull[m]);
       }
       __syncwarp();
@@ -278,7 +286,10 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
       const int m = mi % kMetaRing;
       if (!mbar_wait(&mhead[m], (mi / kMetaRing) & 1, abort, p.err)) break;
       if (s_meta[m].end) {
-        if (lane == 0) mbar_arrive(&mfull[m]);
+        if (lane == 0) {
+          mbar_arrive(&mrows[m]);
+          mbar_arrive(&mfull[m]);
+        }
         break;
       }
       const int j = s_meta[m].j, tt = s_meta[m].tt, rg = s_meta[m].rg;
@@ -286,11 +297,15 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
       const int T = sl.y, q0 = sl.z, rows = s_ucnt[j];
       const int nt = min(kTileTok, T - tt * kTileTok);
       const int qt = q0 + tt * kTileTok;
-      // row of this lane (lanes 0..15) and token of this lane (lanes 0..7)
+      // row of this lane (lanes 0..15) and token of this lane (lanes 0..7); the rows go out
+      // first (mrows: all the copier needs), the coefficients after one more round trip
       const int ridx = rg * kTileRows + (lane & 15);
       const int n_l = __ldcg(&p.ulist[(size_t)j * Imax + (ridx < rows ? ridx : rg * kTileRows)]);
       const int tok_l = lane < nt ? __ldcg(&p.pair_token[qt + lane]) : -1;
       const float w_l = lane < nt ? __ldcg(&p.pair_w[qt + lane]) : 0.f;
+      if (lane < kTileRows) s_meta[m].rows[lane] = n_l;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&mrows[m]);
       // coefficients: lane l covers row l/2, columns 4*(l&1) .. +3
       const int r = lane >> 1, c0 = (lane & 1) * 4;
       const int n = __shfl_sync(0xffffffffu, n_l, r);
@@ -307,7 +322,6 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
 #pragma unroll
       for (int c = 0; c < 4; ++c)
         s_meta[m].coef[r][c0 + c] = ((bits[c] >> (n & 31)) & 1u) ? av[c] : 0.f;
-      if (lane < kTileRows) s_meta[m].rows[lane] = n_l;
       if (lane < kTileTok) {
         s_meta[m].tok[lane] = tok_l;
         s_meta[m].w[lane] = w_l;
@@ -324,7 +338,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
     int it = 0;
     for (int mi = 0; !*abort; ++mi) {
       const int m = mi % kMetaRing;
-      if (!mbar_wait(&mfull[m], (mi / kMetaRing) & 1, abort, p.err)) break;
+      if (!mbar_wait(&mrows[m], (mi / kMetaRing) & 1, abort, p.err)) break;
       if (s_meta[m].end) break;
       const __nv_bfloat16* row = s_meta[m].ud + (size_t)s_meta[m].rows[lane & 15] * 2 * H;
       __syncwarp();

@@ -85,6 +85,7 @@ def test_forward_rejects_null_handle(lib):
     assert lib.moe_destroy(None) == moe.MOE_OK
     assert lib.moe_debug_lists(None, 1, None, None, None, None, None, None, None) == \
         moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_set_dense_min_tokens(None, 8) == moe.MOE_ERR_INVALID_ARG
 
 
 def test_status_strings(lib):

@@ -7,11 +7,13 @@ import torch
 
 import oracle
 import synth
-from sparse_expert_ffn_logits_b200 import (MOE_ERR_DEVICE, MOE_OK, moe_get_error)
+from sparse_expert_ffn_logits_b200 import (MOE_ERR_DEVICE, MOE_OK, moe_get_error,
+                                           moe_set_dense_min_tokens)
 from sparse_expert_ffn_logits_b200.workload import DeviceLayer
 from tests import parity
 
 pytestmark = pytest.mark.gpu
+DEFAULT_DENSE_MIN = 48  # the library's default threshold (tokens per expert)
 
 
 def _tokens(dl, B, batch_index):
@@ -215,3 +217,34 @@ def test_llama4_large_batch(llama4):
          shared_weights=shared, expert_cache=cache)
     _run(llama4, 64, ("topk", 0.5), ("topk", 0.5), batch_index=98, tokens=[1, 33, 63],
          shared_weights=shared, expert_cache=cache)
+
+
+# ---------------------------------------------------------------------------------------------
+# the dense masked path on the tensor cores (experts with >= dense_min tokens), forced on
+@pytest.mark.parametrize("s", [0.0, 0.9])
+def test_olmoe_dense_path(olmoe, s):
+    moe_set_dense_min_tokens(olmoe.h, 1)
+    try:
+        _run(olmoe, 64, ("topk", s), batch_index=60 + int(10 * s), tokens=np.arange(0, 64, 3))
+        _run(olmoe, 256, ("topk", 0.5), batch_index=70, tokens=np.arange(5, 256, 25))
+    finally:
+        moe_set_dense_min_tokens(olmoe.h, DEFAULT_DENSE_MIN)
+
+
+def test_dsv2l_mixed_paths(dsv2l):
+    # shared experts (T = B = 16) dense, routed experts (T ~ 1.5) sparse
+    moe_set_dense_min_tokens(dsv2l.h, 16)
+    try:
+        _run(dsv2l, 16, ("topk", 0.9), ("topk", 0.5), batch_index=80)
+        _run(dsv2l, 64, ("topk", 0.5), ("topk", 0.0), batch_index=81, tokens=np.arange(0, 64, 5))
+    finally:
+        moe_set_dense_min_tokens(dsv2l.h, DEFAULT_DENSE_MIN)
+
+
+def test_gptoss_dense_partial_tiles(gptoss):
+    # H = I = 2880: the last 128-row tile of every GEMM is partial
+    moe_set_dense_min_tokens(gptoss.h, 1)
+    try:
+        _run(gptoss, 32, ("topk", 0.9), batch_index=90, tokens=np.arange(0, 32, 4))
+    finally:
+        moe_set_dense_min_tokens(gptoss.h, DEFAULT_DENSE_MIN)
