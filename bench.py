@@ -28,6 +28,7 @@ sys.path.insert(0, ROOT)
 METRIC = "MoE-layer decode tokens/sec and HBM GB/s vs roofline at batch 1–256, sparsity 0/50/90%"
 UNIT = "tokens/s"
 FALLBACK_HBM_GBS = 6650.0
+DEFAULT_DENSE_MIN = -1  # the library's default: automatic path choice per call
 
 
 def parse():
@@ -43,6 +44,9 @@ def parse():
     ap.add_argument("--no-sweep", dest="sweep", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target host time of the oracle sample")
+    ap.add_argument("--crossover", action="store_true",
+                    help="time the sparse kernels against the tensor-core path per batch size "
+                         "(one GPU) and print the table instead of the benchmark line")
     return ap.parse_args()
 
 
@@ -428,6 +432,56 @@ def run_reference(args):
                     "d2h_bytes_per_step": 0}}
 
 
+def run_crossover(args):
+    """Layer time per batch size with the dense tensor-core path off (every expert sparse) and
+    forced on (every expert dense), L2 flushed before each call; prints one JSON line per
+    (batch, sparsity) and a summary with the smallest batch at which the dense path wins."""
+    import torch
+
+    import synth
+    from sparse_expert_ffn_logits_b200 import moe_set_dense_min_tokens
+    from sparse_expert_ffn_logits_b200.workload import DeviceLayer
+    shape = synth.SHAPES[args.workload]
+    batches = [b for b in (8, 16, 32, 64, 128, 256)]
+    dl = DeviceLayer(shape, max_tokens=max(batches))
+    default_min = DEFAULT_DENSE_MIN
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    flush_w = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device="cuda")
+    flush_r = torch.ones_like(flush_w)
+    rows = []
+    for B in batches:
+        xs = [dl.tokens(B, synth.token_seed(shape, 500 + i)) for i in range(8)]
+        out = torch.empty_like(xs[0])
+        for s in (0.0, 0.5, 0.9):
+            rule = ("topk", s)
+            t = {}
+            for name, dmin in (("sparse", 0), ("dense", 1), ("auto", default_min)):
+                moe_set_dense_min_tokens(dl.h, dmin)
+                for i in range(3):
+                    dl.forward(xs[i], rule, rule, out=out)
+                ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                      for _ in range(args.steps)]
+                for i in range(args.steps):
+                    flush_w.zero_()
+                    flush_r.sum()
+                    ev[i][0].record()
+                    dl.forward(xs[i % len(xs)], rule, rule, out=out)
+                    ev[i][1].record()
+                torch.cuda.synchronize()
+                t[name] = statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3
+            row = {"workload": shape.name, "batch": B, "sparsity": s,
+                   "tokens_per_expert": round(B * shape.top_k / shape.n_routed, 2),
+                   "sparse_us": round(t["sparse"], 1), "dense_us": round(t["dense"], 1),
+                   "auto_us": round(t["auto"], 1),
+                   "faster": "dense" if t["dense"] < t["sparse"] else "sparse"}
+            rows.append(row)
+            print(json.dumps(row), flush=True)
+    dl.close()
+    wins = [r["batch"] for r in rows if r["faster"] == "dense"]
+    print(json.dumps({"workload": shape.name, "crossover_batch": min(wins) if wins else None,
+                      "rows": len(rows)}))
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -436,6 +490,9 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
+        return 0
+    if args.crossover:
+        run_crossover(args)
         return 0
     import torch
     import torch.distributed as dist

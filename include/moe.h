@@ -170,14 +170,20 @@ moe_status moe_read_trace(moe_handle* h, unsigned long long* host, size_t n);
  * MOE_OK with *device_code = 0. */
 moe_status moe_get_error(moe_handle* h, int* device_code);
 
-/* Path choice per expert.  An expert (routed or shared) that receives at least min_tokens tokens
- * in a call is computed by the dense masked path on the tensor cores (gate GEMM, the same
- * selection, up GEMM times the 0/1 mask and SiLU(g), down GEMM), the others by the sparse
- * kernels; both compute the same function ("Uncovering Intra-expert Activation Sparsity ...",
- * technical summary, Methodology: sparse or dense kernels chosen by batch size).  min_tokens = 0
- * turns the dense path off; bf16 layers only (fp32 layers always take the sparse kernels).
- * The default comes from the crossover measured on B200.  INVALID_ARG for a NULL handle or a
- * negative count.  Takes effect from the next moe_forward. */
+/* Path choice.  Both paths compute the same function ("Uncovering Intra-expert Activation
+ * Sparsity ...", technical summary, Methodology: sparse or dense kernels chosen by batch size):
+ * the sparse kernels read only the kept neurons' rows; the dense masked path runs the gate, up and
+ * down projections as tcgen05 GEMMs, keeps the same neurons and multiplies the up projection by
+ * the 0/1 mask and SiLU(g).  bf16 layers only (fp32 layers always take the sparse kernels).
+ *   MOE_DENSE_AUTO (-1, the default)  per call: every expert takes the dense path when the
+ *                      batch's average tokens per routed expert n_tokens * top_k / n_routed is
+ *                      >= 6 (>= 10 when the routed sparsity is above 0.7), else the sparse path;
+ *                      thresholds measured on B200
+ *   0                  never the dense path
+ *   n > 0              per expert: an expert (routed or shared) with >= n tokens in the call
+ *                      takes the dense path, the others the sparse kernels
+ * INVALID_ARG for a NULL handle or a value below -1.  Takes effect from the next moe_forward. */
+#define MOE_DENSE_AUTO (-1)
 moe_status moe_set_dense_min_tokens(moe_handle* h, int min_tokens);
 
 /* Frees the workspace and the handle (synchronises the device first).  NULL is a no-op. */

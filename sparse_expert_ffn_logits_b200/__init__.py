@@ -207,8 +207,12 @@ def moe_get_error(h):
     return rc, code.value
 
 
+MOE_DENSE_AUTO = -1
+
+
 def moe_set_dense_min_tokens(h, min_tokens):
-    """Experts with at least min_tokens tokens take the tensor-core path (0: never)."""
+    """Path choice: MOE_DENSE_AUTO (per call, the default), 0 (never dense) or a per-expert
+    token threshold (see include/moe.h)."""
     _check(_lib().moe_set_dense_min_tokens(ctypes.c_void_p(h) if h else None, int(min_tokens)),
            "moe_set_dense_min_tokens")
 

@@ -317,16 +317,21 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
             }
           }
         } else if (kMode == 1) {
+          // every load of the chunk first (they are independent), then the products and stores
+          uint32_t bits[32];
+          float a[32];
+          const bool live = row < r.mext;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const size_t q = (size_t)(r.q0 + r.n0 + c0 + min(c, nc - 1));
+            bits[c] = live ? __ldcg(&p.maskbits[q * (p.Imax / 32) + (row >> 5)]) : 0u;
+            a[c] = live ? __ldcg(&p.act[q * p.Imax + row]) : 0.f;
+          }
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             if (c >= nc) continue;
             const size_t q = (size_t)(r.q0 + r.n0 + c0 + c);
-            float h = 0.f;
-            if (row < r.mext) {
-              const uint32_t bits = __ldcg(&p.maskbits[q * (p.Imax / 32) + (row >> 5)]);
-              if ((bits >> (row & 31)) & 1u) h = __ldcg(&p.act[q * p.Imax + row]) *
-                                                __uint_as_float(v[c]);
-            }
+            const float h = ((bits[c] >> (row & 31)) & 1u) ? a[c] * __uint_as_float(v[c]) : 0.f;
             p.hbuf[q * p.imax_pad + row] = __float2bfloat16_rn(h);
           }
         } else {
