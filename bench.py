@@ -148,6 +148,27 @@ def traffic_of(key):
     return ent["bytes"] if h.hexdigest()[:16] == ent["source_sha"] else None
 
 
+def job_time_ms(local_ms, world, device):
+    """The job's time: the largest of the ranks' device-timed totals (every rank calls this)."""
+    if world == 1:
+        return local_ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([local_ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, batch, steps, job_ms):
+    """Tokens per second of the whole job: every rank processed `steps` batches of `batch`."""
+    return world * batch * steps / (job_ms / 1e3)
+
+
+def token_stream(rank, i):
+    """Index of rank `rank`'s i-th token batch: ranks draw disjoint streams (i < 1000)."""
+    return rank * 1000 + i
+
+
 def run_cuda(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -169,7 +190,7 @@ def run_cuda(args, rank, world, local_rank):
     pool_n = 32
 
     def pool(nb):
-        return [dl.tokens(nb, synth.token_seed(shape, rank * 1000 + i)) for i in range(pool_n)]
+        return [dl.tokens(nb, synth.token_seed(shape, token_stream(rank, i))) for i in range(pool_n)]
 
     xs = pool(B)
     out = torch.empty_like(xs[0])
@@ -228,12 +249,8 @@ def run_cuda(args, rank, world, local_rank):
     torch.cuda.synchronize()
     clock_info = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in evs]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    value = world * B * args.steps / (total_ms / 1e3)
+    total_ms = job_time_ms(sum(step_ms), world, dev)
+    value = job_throughput(world, B, args.steps, total_ms)
 
     # ---- per-stage durations (kernels launched back to back, events between them)
     stage_evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)]
@@ -289,13 +306,9 @@ def run_cuda(args, rank, world, local_rank):
         moe_forward_host(dl.h, xh[i % 8], B, dl.router, dl.routed, dl.shared, sr, ss, oh)
         e2e_ev[i][1].record()
     torch.cuda.synchronize()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = job_time_ms(sum(a.elapsed_time(b) for a, b in e2e_ev), world, dev)
     io_bytes = B * shape.hidden * shape.elt
-    e2e = {"value": round(world * B * args.steps / (e2e_ms / 1e3), 1), "unit": UNIT,
+    e2e = {"value": round(job_throughput(world, B, args.steps, e2e_ms), 1), "unit": UNIT,
            "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes,
            "api": "moe_forward_host"}
 

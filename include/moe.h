@@ -38,7 +38,7 @@ typedef enum {
   MOE_ERR_OOM = 3,         /* the workspace allocation failed */
   MOE_ERR_CUDA = 4,        /* a CUDA call or launch failed */
   MOE_ERR_DEVICE = 5,      /* the kernels set the device error word (moe_get_error) */
-  MOE_ERR_TIMEOUT = 6      /* reserved for bounded waits; no entry point returns it yet */
+  MOE_ERR_TIMEOUT = 6      /* a bounded wait inside a kernel gave up (moe_get_error) */
 } moe_status;
 
 typedef enum { MOE_BF16 = 0, MOE_F32 = 1 } moe_dtype;
@@ -165,10 +165,16 @@ moe_status moe_profile_stages(moe_handle* h, void* const* events, int n_events);
 moe_status moe_read_trace(moe_handle* h, unsigned long long* host, size_t n);
 
 /* Synchronises the device, reads and clears the device error word.  Returns MOE_ERR_DEVICE
- * (code in *device_code: 1 = NaN router logit, 2 = NaN activation, 3 = a bounded wait inside a
- * kernel gave up after 0.2 s; the output of that call is then invalid) if it was set, else
- * MOE_OK with *device_code = 0. */
+ * (code in *device_code: 1 = NaN router logit, 2 = NaN activation) or MOE_ERR_TIMEOUT (code 3:
+ * a bounded wait inside a kernel gave up after 0.2 s; the output of that call is then invalid)
+ * if it was set, else MOE_OK with *device_code = 0. */
 moe_status moe_get_error(moe_handle* h, int* device_code);
+
+/* Failure-detection test hook (the paper has none): launches one warp that waits, with the
+ * kernels' own bounded wait, on a barrier that nothing completes.  After the wait's 0.2 s limit
+ * it records a timeout in the handle's error word and returns; the GPU context stays usable and
+ * the next moe_get_error returns MOE_ERR_TIMEOUT.  Asynchronous on `stream`. */
+moe_status moe_debug_force_timeout(moe_handle* h, void* stream);
 
 /* Path choice.  Both paths compute the same function ("Uncovering Intra-expert Activation
  * Sparsity ...", technical summary, Methodology: sparse or dense kernels chosen by batch size):

@@ -51,7 +51,8 @@ _LIB = None
 # C entry points declared in include/moe.h
 EXPORTS = ("moe_create", "moe_packed_bytes", "moe_pack_experts", "moe_forward",
            "moe_forward_host", "moe_debug_lists", "moe_profile_stages", "moe_read_trace",
-           "moe_get_error", "moe_set_dense_min_tokens", "moe_destroy", "moe_route_noalloc",
+           "moe_get_error", "moe_debug_force_timeout", "moe_set_dense_min_tokens", "moe_destroy",
+           "moe_route_noalloc",
            "moe_status_string")
 MOE_STAGE_EVENTS = 6
 STAGES = ("router", "gate", "select", "updown", "finalize")
@@ -80,6 +81,7 @@ def _lib():
         lib.moe_get_error.argtypes = [P, ctypes.POINTER(I)]
         lib.moe_destroy.argtypes = [P]
         lib.moe_set_dense_min_tokens.argtypes = [P, I]
+        lib.moe_debug_force_timeout.argtypes = [P, P]
         lib.moe_route_noalloc.argtypes = [ctypes.POINTER(MoEConfig), P, I, P, P, P, P]
         lib.moe_status_string.argtypes = [I]
         lib.moe_status_string.restype = ctypes.c_char_p
@@ -199,15 +201,22 @@ def moe_read_trace(h):
 
 
 def moe_get_error(h):
-    """(status, device_code); status is MOE_OK or MOE_ERR_DEVICE (does not raise for those)."""
+    """(status, device_code); status is MOE_OK, MOE_ERR_DEVICE or MOE_ERR_TIMEOUT (does not
+    raise for those)."""
     code = ctypes.c_int(0)
     rc = _lib().moe_get_error(ctypes.c_void_p(h), ctypes.byref(code))
-    if rc not in (MOE_OK, MOE_ERR_DEVICE):
+    if rc not in (MOE_OK, MOE_ERR_DEVICE, MOE_ERR_TIMEOUT):
         raise MoEError(rc, "moe_get_error")
     return rc, code.value
 
 
 MOE_DENSE_AUTO = -1
+
+
+def moe_debug_force_timeout(h, stream=None):
+    """Test hook: a bounded wait that runs out (see include/moe.h)."""
+    _check(_lib().moe_debug_force_timeout(ctypes.c_void_p(h) if h else None, _stream(stream)),
+           "moe_debug_force_timeout")
 
 
 def moe_set_dense_min_tokens(h, min_tokens):

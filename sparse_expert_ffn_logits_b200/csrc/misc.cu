@@ -1,5 +1,6 @@
 // misc.cu - output cast, weight packing, debug export and per-handle kernel configuration.
 #include "kernels.h"
+#include "tma.cuh"
 
 namespace moe {
 
@@ -92,6 +93,28 @@ cudaError_t launch_pack_down(const void* w_down, void* packed_updown, int n, int
   else
     pack_down_kernel<float><<<grid, block, 0, st>>>(static_cast<const float*>(w_down),
                                                     static_cast<float*>(packed_updown), I, H);
+  return cudaGetLastError();
+}
+
+// Failure-detection hook: one warp waits, with the same bounded wait as the ring kernels, on an
+// mbarrier that nothing ever completes.  The wait gives up after its time limit, sets the error
+// word (timeout) and the kernel returns: the path that a stalled pipeline takes, exercised
+// without a stalled pipeline.
+__global__ void force_timeout_kernel(FwdParams p) {
+  __shared__ uint64_t bar;
+  __shared__ int s_abort;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    s_abort = 0;
+    mbar_init_fence();
+  }
+  __syncwarp();
+  volatile int* abort = &s_abort;
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, abort, p.err);  // phase 0 never completes
+}
+
+cudaError_t launch_force_timeout(const FwdParams& p, cudaStream_t st) {
+  force_timeout_kernel<<<1, 32, 0, st>>>(p);
   return cudaGetLastError();
 }
 

@@ -20,6 +20,7 @@
 
 #include "../../include/moe.h"
 #include "kernels.h"
+#include "tma.cuh"
 
 using moe::FwdParams;
 using moe::LaunchShape;
@@ -429,7 +430,12 @@ moe_status moe_get_error(moe_handle* h, int* device_code) {
   if (v == 0) return MOE_OK;
   *device_code = v;
   if (cudaMemset(h->base.err, 0, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
-  return MOE_ERR_DEVICE;
+  return v == moe::kErrTimeout ? MOE_ERR_TIMEOUT : MOE_ERR_DEVICE;
+}
+
+moe_status moe_debug_force_timeout(moe_handle* h, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  return cuda_status(moe::launch_force_timeout(h->base, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_set_dense_min_tokens(moe_handle* h, int min_tokens) {

@@ -19,6 +19,8 @@
 namespace moe {
 namespace {
 
+constexpr size_t kRouterClusterPartBytes = 64 * 1024;  // partial logits of one cluster CTA
+
 // Order key of (logit, expert): larger key = larger logit, then lower expert index; 0 = none.
 __device__ __forceinline__ unsigned long long topk_key(float v, int e) {
   uint32_t u = __float_as_uint(v);
@@ -330,6 +332,108 @@ __global__ void __launch_bounds__(kThreads) router_kernel(FwdParams p) {
   trace_point(p.trace, 0, 6);
 }
 
+// ---- single-cluster variant for small batches ------------------------------------------------
+// One thread-block cluster does the whole step: CTA r of the C CTAs computes the partial logits
+// of every (expert, token) over the r-th slice of H into its own shared memory; after a cluster
+// barrier each CTA sums, for its tokens (t = r, r + C, ...), the C partials in rank order through
+// distributed shared memory, picks the top-k; after a second barrier CTA 0 groups the pairs.
+// No global tickets, no fences between CTAs of different SMs' L1s, no second wave of loads.
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_size() {
+  uint32_t n;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(n));
+  return n;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
+}
+// f32 at the same shared-memory offset as `local`, in the shared memory of cluster CTA `rank`
+// (no ordering constraint of its own: the cluster barrier before the reads orders them)
+__device__ __forceinline__ float ld_dsmem(const float* local, uint32_t rank) {
+  uint32_t ra;
+  asm("mapa.shared::cluster.u32 %0, %1, %2;"
+      : "=r"(ra)
+      : "r"((uint32_t)__cvta_generic_to_shared(local)), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra));
+  return v;
+}
+constexpr int kMaxClusterCtas = 16;
+
+template <typename T, int PER>
+__global__ void __launch_bounds__(kThreads) router_cluster_kernel(FwdParams p) {
+  extern __shared__ uint32_t dyn[];  // partial logits [B][E], later group_pairs' scratch
+  __shared__ const T* s_xt[kWarps][kTileTok];
+  __shared__ unsigned long long scratch[33];
+  __shared__ float s_lg[kWarps][kMaxRouted];
+  __shared__ float s_tv[kWarps][kMaxTopK];
+  __shared__ int s_ti[kWarps][kMaxTopK];
+  trace_point(p.trace, 0, 0);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
+  const uint32_t rank = cluster_rank(), C = cluster_size();
+  const int H = p.H, E = p.E, B = p.B;
+  const int nblk = H / 32;
+  const int blo = (int)(rank * nblk / C), bhi = (int)((rank + 1) * nblk / C);
+  const T* x = static_cast<const T*>(p.x);
+  const T* wr = static_cast<const T*>(p.router);
+  float* part = reinterpret_cast<float*>(dyn);
+  const int etiles = (E + kTileRows - 1) / kTileRows, ttiles = (B + kTileTok - 1) / kTileTok;
+  for (int tile = warp; tile < etiles * ttiles; tile += kWarps) {
+    const int e0 = (tile % etiles) * kTileRows, t0 = (tile / etiles) * kTileTok;
+    if (lane < kTileTok) s_xt[warp][lane] = t0 + lane < B ? x + (size_t)(t0 + lane) * H : nullptr;
+    __syncwarp();
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+    tile_dot<4>(wr + (size_t)min(e0 + g, E - 1) * H, wr + (size_t)min(e0 + g + 8, E - 1) * H,
+                s_xt[warp], blo, 1, bhi, d);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int e = e0 + g + (c >> 1) * 8, tok = t0 + 2 * t + (c & 1);
+      if (e < E && tok < B) part[tok * E + e] = d[c];
+    }
+    __syncwarp();
+  }
+  trace_point(p.trace, 0, 1);
+  cluster_sync_all();
+  trace_point(p.trace, 0, 2);
+  bool nan_seen = false;
+  for (int i = warp;; i += kWarps) {
+    const int tok = (int)rank + (int)C * i;
+    if (tok >= B) break;
+    for (int e = lane; e < E; e += 32) {
+      float pv[kMaxClusterCtas];  // every rank's partial in flight, then summed in rank order
+#pragma unroll
+      for (uint32_t r = 0; r < kMaxClusterCtas; ++r)
+        pv[r] = r < C ? ld_dsmem(&part[tok * E + e], r) : 0.f;
+      float v = 0.f;
+#pragma unroll
+      for (int r = 0; r < kMaxClusterCtas; ++r) v += pv[r];
+      s_lg[warp][e] = v;
+      p.logits[(size_t)tok * E + e] = v;
+      nan_seen |= isnan(v);
+    }
+    __syncwarp();
+    topk_token<PER>(p, tok, s_lg[warp], s_tv[warp], s_ti[warp]);
+    __syncwarp();
+  }
+  if (nan_seen) set_error(p.err, kErrNanLogit);
+  trace_point(p.trace, 0, 3);
+  __threadfence();
+  cluster_sync_all();  // every top-k is written; no CTA reads another's shared memory after this
+  if (rank == 0) {
+    trace_point(p.trace, 0, 5);
+    group_pairs(p, dyn, scratch);
+    trace_point(p.trace, 0, 6);
+  }
+}
+
+int g_router_cluster = 0;  // CTAs of the single-cluster router (0: not available)
+
 }  // namespace
 
 size_t router_smem_bytes(int E, int B) {
@@ -358,7 +462,43 @@ cudaError_t launch_router_t(const FwdParams& p, dim3 grid, size_t smem, cudaStre
   return launch_pdl(router_kernel<T, 16>, grid, dim3(kThreads), smem, st, false, p);
 }
 
+// The single-cluster router holds the batch's partial logits in each CTA's shared memory.
+bool router_uses_cluster(int E, int B) {
+  return g_router_cluster > 0 && (size_t)E * B * 4 <= kRouterClusterPartBytes;
+}
+
+template <typename T, int PER>
+cudaError_t launch_router_cluster_t(const FwdParams& p, size_t smem, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(g_router_cluster);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = g_router_cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, router_cluster_kernel<T, PER>, p);
+}
+
+template <typename T>
+cudaError_t launch_router_cluster(const FwdParams& p, cudaStream_t st) {
+  const size_t part = (size_t)p.E * p.B * 4, grp = router_smem_bytes(p.E, p.B);
+  const size_t smem = part > grp ? part : grp;
+  if (p.E <= 32) return launch_router_cluster_t<T, 1>(p, smem, st);
+  if (p.E <= 64) return launch_router_cluster_t<T, 2>(p, smem, st);
+  if (p.E <= 128) return launch_router_cluster_t<T, 4>(p, smem, st);
+  if (p.E <= 256) return launch_router_cluster_t<T, 8>(p, smem, st);
+  return launch_router_cluster_t<T, 16>(p, smem, st);
+}
+
 cudaError_t launch_router(const FwdParams& p, int dtype, cudaStream_t st) {
+  if (router_uses_cluster(p.E, p.B))
+    return dtype == 0 ? launch_router_cluster<__nv_bfloat16>(p, st)
+                      : launch_router_cluster<float>(p, st);
   dim3 grid(((p.E + kTileRows - 1) / kTileRows) * p.hsplit, (p.B + kTileTok - 1) / kTileTok);
   const size_t smem = router_smem_bytes(p.E, p.B);
   if (dtype == 0) return launch_router_t<__nv_bfloat16>(p, grid, smem, st);
@@ -375,10 +515,58 @@ cudaError_t configure_router_t(int budget) {
   return e;
 }
 
+template <typename T>
+cudaError_t configure_router_cluster_t(int budget, bool wide) {
+  cudaError_t e = cudaSuccess;
+  auto one = [&](auto kernel) {
+    if (e != cudaSuccess) return;
+    e = allow_max_smem(kernel, budget);
+    if (e == cudaSuccess && wide)
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  };
+  one(router_cluster_kernel<T, 1>);
+  one(router_cluster_kernel<T, 2>);
+  one(router_cluster_kernel<T, 4>);
+  one(router_cluster_kernel<T, 8>);
+  one(router_cluster_kernel<T, 16>);
+  return e;
+}
+
 cudaError_t configure_router(int budget) {
   cudaError_t e = configure_router_t<__nv_bfloat16>(budget);
   if (e != cudaSuccess) return e;
-  return configure_router_t<float>(budget);
+  e = configure_router_t<float>(budget);
+  if (e != cudaSuccess) return e;
+  // single-cluster router: 16 CTAs where the device takes a cluster that wide, else 8
+  if (g_router_cluster == 0) {
+    int c = 0;
+    for (int want : {16, 8}) {
+      if (configure_router_cluster_t<__nv_bfloat16>(budget, want > 8) != cudaSuccess ||
+          configure_router_cluster_t<float>(budget, want > 8) != cudaSuccess)
+        continue;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(want);
+      cfg.blockDim = dim3(kThreads);
+      cfg.dynamicSmemBytes = kRouterClusterPartBytes;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = want;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, router_cluster_kernel<__nv_bfloat16, 16>, &cfg) ==
+              cudaSuccess &&
+          n > 0) {
+        c = want;
+        break;
+      }
+    }
+    cudaGetLastError();  // a refused cluster width is not an error of this call
+    g_router_cluster = c;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace moe

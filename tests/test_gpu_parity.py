@@ -7,7 +7,8 @@ import torch
 
 import oracle
 import synth
-from sparse_expert_ffn_logits_b200 import (MOE_ERR_DEVICE, MOE_OK, moe_get_error,
+from sparse_expert_ffn_logits_b200 import (MOE_ERR_DEVICE, MOE_ERR_TIMEOUT, MOE_OK,
+                                           moe_debug_force_timeout, moe_get_error,
                                            moe_set_dense_min_tokens)
 from sparse_expert_ffn_logits_b200.workload import DeviceLayer
 from tests import parity
@@ -118,6 +119,16 @@ def test_zero_tokens_and_errors(tiny):
     tiny.forward(xd, ("topk", 0.5))
     st, code = moe_get_error(tiny.h)
     assert st == MOE_ERR_DEVICE and code in (1, 2)
+    st, code = moe_get_error(tiny.h)
+    assert st == MOE_OK and code == 0
+    _run(tiny, 4, ("topk", 0.5))
+
+
+def test_bounded_wait_reports_timeout(tiny):
+    """A wait that nothing ends gives up after its limit and reports, the GPU stays usable."""
+    moe_debug_force_timeout(tiny.h)
+    st, code = moe_get_error(tiny.h)
+    assert st == MOE_ERR_TIMEOUT and code == 3
     st, code = moe_get_error(tiny.h)
     assert st == MOE_OK and code == 0
     _run(tiny, 4, ("topk", 0.5))
