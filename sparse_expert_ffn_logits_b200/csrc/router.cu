@@ -374,6 +374,7 @@ __global__ void __launch_bounds__(kThreads) router_cluster_kernel(FwdParams p) {
   __shared__ float s_lg[kWarps][kMaxRouted];
   __shared__ float s_tv[kWarps][kMaxTopK];
   __shared__ int s_ti[kWarps][kMaxTopK];
+  pdl_trigger();  // the gate kernel may start its prologue now
   trace_point(p.trace, 0, 0);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
   const uint32_t rank = cluster_rank(), C = cluster_size();

@@ -25,7 +25,6 @@ constexpr int kSelWarps = kSelThreads / 32;
 __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
   extern __shared__ uint32_t sm[];
   __shared__ int hist[2 * kSelWarps * 8];
-  __shared__ int scratch[33];
   __shared__ uint32_t cbuf[32];
   __shared__ int s_ncand, s_need, s_last;
   __shared__ uint32_t s_tau;
@@ -255,31 +254,32 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
     }
     __syncthreads();
     if (q == (int)blockIdx.x) trace_point(p.trace, 2, 6);
-    if (s_last) {
-      // last pair of this expert: compact the union bitmask into a row list, clear it
+    if (s_last && warp == 0) {
+      // last pair of this expert: warp 0 compacts the union bitmask into the ascending row
+      // list (lane l takes a contiguous block of words) and clears it
       __threadfence();
-      const int W = I / 32;
-      const int per = (W + blockDim.x - 1) / blockDim.x;
-      const int wb = min(W, (int)threadIdx.x * per), we = min(W, wb + per);
-      uint32_t words[2];
+      const int W = I / 32, wpl = (W + 31) / 32;
+      const int wb = min(W, lane * wpl), we = min(W, wb + wpl);
       int c = 0;
-      for (int w = wb; w < we; ++w) {
-        words[w - wb] = __ldcg(&urow[w]);
-        c += __popc(words[w - wb]);
+      for (int w = wb; w < we; ++w) c += __popc(__ldcg(&urow[w]));
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
       }
-      int utotal;
-      int upos = block_exclusive_scan(c, scratch, &utotal);
+      int upos = incl - c;
       int* ul = p.ulist + (size_t)j * Imax;
       for (int w = wb; w < we; ++w) {
-        uint32_t b = words[w - wb];
+        uint32_t b = __ldcg(&urow[w]);
+        urow[w] = 0;
         while (b) {
           ul[upos++] = w * 32 + __ffs(b) - 1;
           b &= b - 1;
         }
-        urow[w] = 0;
       }
-      if (threadIdx.x == 0) {
-        p.ucnt[j] = utotal;
+      if (lane == 31) {
+        p.ucnt[j] = incl;
         p.slot_ticket[j] = 0;
       }
     }

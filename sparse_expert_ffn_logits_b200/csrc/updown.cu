@@ -304,6 +304,10 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
       const int tok_l = lane < nt ? __ldcg(&p.pair_token[qt + lane]) : -1;
       const float w_l = lane < nt ? __ldcg(&p.pair_w[qt + lane]) : 0.f;
       if (lane < kTileRows) s_meta[m].rows[lane] = n_l;
+      if (lane < kTileTok) {
+        s_meta[m].tok[lane] = tok_l;
+        s_meta[m].w[lane] = w_l;
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&mrows[m]);
       // coefficients: lane l covers row l/2, columns 4*(l&1) .. +3
@@ -322,10 +326,6 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
 #pragma unroll
       for (int c = 0; c < 4; ++c)
         s_meta[m].coef[r][c0 + c] = ((bits[c] >> (n & 31)) & 1u) ? av[c] : 0.f;
-      if (lane < kTileTok) {
-        s_meta[m].tok[lane] = tok_l;
-        s_meta[m].w[lane] = w_l;
-      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&mfull[m]);
     }
@@ -372,7 +372,9 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
   const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(p.x);
   for (int mi = 0;; ++mi) {
     const int m = mi % kMetaRing;
-    mbar_wait(&mfull[m], (mi / kMetaRing) & 1, abort, p.err);
+    // rows, tokens and weights (mrows) are enough for the up projection; the coefficients
+    // (mfull, one more L2 round trip) are awaited before the epilogue
+    mbar_wait(&mrows[m], (mi / kMetaRing) & 1, abort, p.err);
     // the end (or an abort) is decided by all consumer warps together
     if (consumer_sync_or(kThreads, s_meta[m].end || *abort)) {
       trace_value(p.trace, 3, 5, (unsigned long long)mi);
@@ -447,6 +449,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
     if (!kReg && lane == 0 && xlast) mbar_arrive(&xempty[xb]);
 #pragma unroll
     for (int c = 0; c < 4; ++c) red[ib][warp][c][lane] = d[c];
+    mbar_wait(&mfull[m], (mi / kMetaRing) & 1, abort, p.err);
     const int aborted = consumer_sync_or(kThreads, *abort);
     // 2. coefficients times u, rounded to bf16, token-major (one element per thread)
     if (threadIdx.x < 128) {
