@@ -16,6 +16,7 @@ constexpr int kMaxShared = 8;
 constexpr int kMaxRouted = 512;
 constexpr int kMaxTokens = 1024;
 constexpr int kMaxHsplit = 16;     // router slices of H
+constexpr int kMaxI = 16384;       // largest intermediate size
 
 // device error word codes
 constexpr int kErrNanLogit = 1;
@@ -86,10 +87,8 @@ struct FwdParams {
   unsigned* slot_ticket;   // [E+S]
   float* act;          // [Pmax][Imax]
   uint32_t* maskbits;  // [Pmax][Imax/32]
-  int* lists;          // [Pmax][Imax]
-  int* cnt;            // [Pmax]
   uint32_t* ubits;     // [E+S][Imax/32]
-  int* ulist;          // [E+S][Imax]
+  int* ulist;          // [E+S][Imax] ascending union rows of each slot
   int* ucnt;           // [E+S]
   float* out_acc;      // [Bmax][H]
   int* err;            // device error word

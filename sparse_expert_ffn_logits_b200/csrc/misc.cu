@@ -55,19 +55,45 @@ __global__ void pack_down_kernel(const T* __restrict__ wd, T* __restrict__ ud, i
   }
 }
 
-// Reorders the per-pair lists / counts / activations of the last call into [token][pair] order.
+// Reorders the last call's per-pair results into [token][pair] order for export: the kept
+// neurons as an ascending index list (from the pair's mask row; -1 after the last) and their
+// count, and the activations.  One CTA per (token, pair); warp 0 writes the list.
 __global__ void debug_gather_kernel(FwdParams p, int* cnt, int* lists, float* act) {
   const int P = p.k + p.S;
   const int tj = blockIdx.x;  // token * P + pair
   const int t = tj / P, jj = tj % P;
   const int q = p.pair_index[t * P + jj];
   const int I = jj < p.k ? p.I : p.Ish;
-  const int c = p.cnt[q];
-  if (threadIdx.x == 0 && cnt) cnt[tj] = c;
-  for (int n = threadIdx.x; n < p.Imax; n += blockDim.x) {
-    if (lists) lists[(size_t)tj * p.Imax + n] = n < c ? p.lists[(size_t)q * p.Imax + n] : -1;
-    if (act) act[(size_t)tj * p.Imax + n] = n < I ? p.act[(size_t)q * p.Imax + n] : 0.f;
+  const int lane = threadIdx.x & 31;
+  const uint32_t* mrow = p.maskbits + (size_t)q * (p.Imax / 32);
+  if (threadIdx.x < 32) {
+    const int W = I / 32, wpl = (W + 31) / 32;
+    const int w0 = min(W, lane * wpl), w1 = min(W, w0 + wpl);
+    int c = 0;
+    for (int w = w0; w < w1; ++w) c += __popc(mrow[w]);
+    int incl = c;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int pos = incl - c;
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    if (lists) {
+      int* out = lists + (size_t)tj * p.Imax;
+      for (int w = w0; w < w1; ++w) {
+        uint32_t b = mrow[w];
+        while (b) {
+          out[pos++] = w * 32 + __ffs(b) - 1;
+          b &= b - 1;
+        }
+      }
+      for (int n = total + lane; n < p.Imax; n += 32) out[n] = -1;
+    }
+    if (lane == 0 && cnt) cnt[tj] = total;
   }
+  if (act)
+    for (int n = threadIdx.x; n < p.Imax; n += blockDim.x)
+      act[(size_t)tj * p.Imax + n] = n < I ? p.act[(size_t)q * p.Imax + n] : 0.f;
 }
 
 }  // namespace

@@ -132,8 +132,6 @@ size_t carve(moe_handle* h, char* base) {
   p.meta = cv.take<int>(moe::kMetaWords);
   p.act = cv.take<float>(Pm * Im);
   p.maskbits = cv.take<uint32_t>(Pm * Wm);
-  p.lists = cv.take<int>(Pm * Im);
-  p.cnt = cv.take<int>(Pm);
   p.ulist = cv.take<int>(slots * Im);
   p.ucnt = cv.take<int>(slots);
   p.err = cv.take<int>(1);

@@ -10,10 +10,10 @@
 //   threshold mode: one pass, keep key > t (the page's single-pass threshold mask).
 // One CTA per pair: its keys sit in shared memory; each radix pass counts digits in registers
 // (packed 16-bit bins), merges them with warp reductions and one barrier.  The kept set is
-// written as an ascending index list + count (for export), as a bitmask row, and
-// OR-ed into the expert's union bitmask.  The last pair of an expert to finish (atomic ticket,
-// no waiting) compacts the union into an ascending row list for the up/down kernel and clears
-// the bitmask.
+// written as the pair's bitmask row and OR-ed into the expert's union bitmask; the last pair
+// of an expert to finish (atomic ticket, no waiting) compacts the union into the ascending row
+// list that the up/down kernel reads, and clears it.  (Ascending index lists and counts of the
+// pairs, for export only, are derived from the mask rows on request.)
 #include "kernels.h"
 
 namespace moe {
@@ -26,7 +26,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
   extern __shared__ uint32_t sm[];
   __shared__ int hist[2 * kSelWarps * 8];
   __shared__ uint32_t cbuf[32];
-  __shared__ int s_ncand, s_need, s_last;
+  __shared__ int s_ncand, s_need, s_eqtot, s_last;
   __shared__ uint32_t s_tau;
   pdl_trigger();
   trace_point(p.trace, 2, 0);
@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
     // routed pairs come first (B * k of them), then the shared experts' pairs
     const int kind = q >= p.B * p.k ? 1 : 0;
     const int I = kind ? p.Ish : p.I;
-    const int j = __ldcg(&p.pair_slot[q]);  // needed only for the union, after the selection
+    const int j = __ldcg(&p.pair_slot[q]);  // the expert's slot, for its union row
     if (threadIdx.x == 0) s_ncand = 0;
     for (int v0 = threadIdx.x;; v0 += 4 * kSelThreads) {
 #pragma unroll
@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
     const float thr = p.sel_t[kind];
     const bool radix = mode == 0 && K > 0 && K < I;
     uint32_t tau = 0;
-    int need = 0;
+    int need = 0, eqtot = 0;  // keys equal to tau, and how many of them are kept
     if (radix) {
       // MSB-first radix select of the K-th largest key, 4-bit digits.  Each thread counts its
       // keys per digit in packed 16-bit fields, a warp sum merges them, and after one barrier
@@ -137,6 +137,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
       if (shift < 0) {
         tau = prefix;  // every bit decided: the krem largest keys equal to prefix are kept
         need = krem;
+        eqtot = cand;
       } else {
         // at most 32 keys carry the prefix: gather them (any order) and rank them in warp 0
         for (int n = threadIdx.x; n < I; n += kSelThreads) {
@@ -161,90 +162,82 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
           if (lane == src) {
             s_tau = mine;
             s_need = krem - gt;
+            s_eqtot = ge - gt;
           }
         }
         __syncthreads();
         tau = s_tau;
         need = s_need;
+        eqtot = s_eqtot;
       }
     }
     if (q == (int)blockIdx.x) trace_point(p.trace, 2, 3);
-    // Kept set, chunk-parallel.  Chunk c = neurons 32c .. 32c + 31 (one ballot each).
-    //   A: every warp takes chunks warp, warp + 8, ...: masks of keys above the cut and equal to
-    //      it (ties exist only in top-K mode).
-    //   B: warp 0 scans the chunks in order: ties are kept lowest index first, so chunk c keeps
-    //      the first min(eq_c, need - ties before c) of its ties; it writes each chunk's kept
-    //      mask and its first list position.
-    //   C: every warp writes its chunks' list entries, mask words and union bits.
+    // Kept set, one ballot per 32-neuron chunk c (neurons 32c .. 32c + 31), written as the
+    // pair's mask row and OR-ed into the expert's union row.  When every key equal to the cut
+    // is kept (the usual case) the mask is simply key >= tau.  Otherwise ties are kept lowest
+    // index first: warp 0 scans the chunks' tie counts in order and trims each chunk's ties.
     const int nch = I / 32;
-    uint32_t* s_km = key + Imax;           // [Imax / 32] above-cut mask, then the kept mask
-    uint32_t* s_em = s_km + Imax / 32;     // [Imax / 32] tie mask
-    int* s_pos = reinterpret_cast<int*>(s_em + Imax / 32);  // [Imax / 32] first list position
-    for (int c = warp; c < nch; c += kSelWarps) {
-      const uint32_t u = key[32 * c + lane];
-      bool above;
-      if (mode == 1) above = __uint_as_float(u) > thr;
-      else if (K >= I) above = true;
-      else if (K == 0) above = false;
-      else above = u > tau;
-      const unsigned gm = __ballot_sync(0xffffffffu, above);
-      const unsigned em = __ballot_sync(0xffffffffu, radix && u == tau);
-      if (lane == 0) {
-        s_km[c] = gm;
-        s_em[c] = em;
-      }
-    }
-    __syncthreads();
-    if (warp == 0) {
-      // lane l owns the contiguous chunk block [l * cpl, (l + 1) * cpl)
-      const int cpl = (nch + 31) / 32;
-      const int c0 = min(nch, lane * cpl), c1 = min(nch, c0 + cpl);
-      int ties = 0;
-      for (int c = c0; c < c1; ++c) ties += __popc(s_em[c]);
-      int tincl = ties;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, tincl, o);
-        if (lane >= o) tincl += y;
-      }
-      int tb = tincl - ties;  // ties before this lane's block
-      int kept = 0;
-      for (int c = c0; c < c1; ++c) {
-        uint32_t em = s_em[c];
-        const int ne = __popc(em);
-        const int take = max(0, min(ne, need - tb));
-        for (int d = ne - take; d > 0; --d) em ^= 1u << (31 - __clz(em));  // drop the highest
-        const uint32_t km = s_km[c] | em;
-        s_km[c] = km;
-        tb += ne;
-        kept += __popc(km);
-      }
-      int kincl = kept;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, kincl, o);
-        if (lane >= o) kincl += y;
-      }
-      int kb = kincl - kept;
-      for (int c = c0; c < c1; ++c) {
-        s_pos[c] = kb;
-        kb += __popc(s_km[c]);
-      }
-      if (lane == 31) p.cnt[q] = kincl;
-    }
-    __syncthreads();
-    int* list = p.lists + (size_t)q * Imax;
     uint32_t* mrow = p.maskbits + (size_t)q * Wmax;
     uint32_t* urow = p.ubits + (size_t)j * Wmax;
-    for (int c = warp; c < nch; c += kSelWarps) {
-      const uint32_t km = s_km[c];
-      if ((km >> lane) & 1u) list[s_pos[c] + __popc(km & lanemask_lt())] = 32 * c + lane;
-      if (lane == 0) {
-        mrow[c] = km;
-        if (km) red_or(&urow[c], km);
+    if (!radix || eqtot == need) {
+      for (int c = warp; c < nch; c += kSelWarps) {
+        const uint32_t u = key[32 * c + lane];
+        bool k_n;
+        if (radix) k_n = u >= tau;
+        else if (mode == 1) k_n = __uint_as_float(u) > thr;
+        else k_n = K >= I;
+        const unsigned km = __ballot_sync(0xffffffffu, k_n);
+        if (lane == 0) {
+          mrow[c] = km;
+          if (km) red_or(&urow[c], km);
+        }
+      }
+    } else {
+      uint32_t* s_km = key + Imax;        // [Imax / 32] above-cut masks, then the kept masks
+      uint32_t* s_em = s_km + Imax / 32;  // [Imax / 32] tie masks
+      for (int c = warp; c < nch; c += kSelWarps) {
+        const uint32_t u = key[32 * c + lane];
+        const unsigned gm = __ballot_sync(0xffffffffu, u > tau);
+        const unsigned em = __ballot_sync(0xffffffffu, u == tau);
+        if (lane == 0) {
+          s_km[c] = gm;
+          s_em[c] = em;
+        }
+      }
+      __syncthreads();
+      if (warp == 0) {
+        const int cpl = (nch + 31) / 32;  // lane l owns chunks [l * cpl, (l + 1) * cpl)
+        const int c0 = min(nch, lane * cpl), c1 = min(nch, c0 + cpl);
+        int ties = 0;
+        for (int c = c0; c < c1; ++c) ties += __popc(s_em[c]);
+        int tincl = ties;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, tincl, o);
+          if (lane >= o) tincl += y;
+        }
+        int tb = tincl - ties;  // ties before this lane's block
+        for (int c = c0; c < c1; ++c) {
+          uint32_t em = s_em[c];
+          const int ne = __popc(em);
+          const int take = max(0, min(ne, need - tb));
+          for (int d = ne - take; d > 0; --d) em ^= 1u << (31 - __clz(em));  // drop the highest
+          s_km[c] |= em;
+          tb += ne;
+        }
+      }
+      __syncthreads();
+      for (int c = warp; c < nch; c += kSelWarps) {
+        if (lane == 0) {
+          const uint32_t km = s_km[c];
+          mrow[c] = km;
+          if (km) red_or(&urow[c], km);
+        }
       }
     }
     if (q == (int)blockIdx.x) trace_point(p.trace, 2, 4);
+    // the last pair of an expert to finish compacts the expert's union (atomic ticket, no
+    // waiting): every pair's union bits are published before its ticket
     __threadfence();
     __syncthreads();
     if (q == (int)blockIdx.x) trace_point(p.trace, 2, 5);
@@ -255,8 +248,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
     __syncthreads();
     if (q == (int)blockIdx.x) trace_point(p.trace, 2, 6);
     if (s_last && warp == 0) {
-      // last pair of this expert: warp 0 compacts the union bitmask into the ascending row
-      // list (lane l takes a contiguous block of words) and clears it
+      // warp 0 compacts the union bitmask into the ascending row list (lane l takes a
+      // contiguous block of words) and clears it
       __threadfence();
       const int W = I / 32, wpl = (W + 31) / 32;
       const int wb = min(W, lane * wpl), we = min(W, wb + wpl);
@@ -283,7 +276,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
         p.slot_ticket[j] = 0;
       }
     }
-    __syncthreads();
+    __syncthreads();  // the next pair reuses the key and chunk buffers
   }
   if (nan_seen) set_error(p.err, kErrNanAct);
   trace_point(p.trace, 2, 7);
@@ -291,8 +284,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
 
 }  // namespace
 
-// keys [Imax] | kept masks, tie masks, list positions [Imax / 32] each
-size_t select_smem_bytes(int imax) { return (size_t)imax * 4 + (size_t)(imax / 32) * 12 + 16; }
+// keys [Imax] | kept masks, tie masks [Imax / 32] each
+size_t select_smem_bytes(int imax) { return (size_t)imax * 4 + (size_t)(imax / 32) * 8 + 16; }
 
 cudaError_t launch_select(const FwdParams& p, const LaunchShape& ls, cudaStream_t st, bool pdl) {
   const int pairs = p.B * (p.k + p.S);
