@@ -259,3 +259,38 @@ def test_gptoss_dense_partial_tiles(gptoss):
         _run(gptoss, 32, ("topk", 0.9), batch_index=90, tokens=np.arange(0, 32, 4))
     finally:
         moe_set_dense_min_tokens(gptoss.h, DEFAULT_DENSE_MIN)
+
+
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("B,dense_min", [(16, DEFAULT_DENSE_MIN), (64, 1)])
+def test_forward_replays_in_a_cuda_graph(olmoe, B, dense_min):
+    """moe_forward allocates nothing and never synchronises: one captured call replays with new
+    token batches (copied into the captured input) and matches eager calls."""
+    moe_set_dense_min_tokens(olmoe.h, dense_min)
+    try:
+        rule = ("topk", 0.9)
+        x_static = olmoe.tokens(B, synth.token_seed(olmoe.shape, 120))
+        out_static = torch.empty_like(x_static)
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            olmoe.forward(x_static, rule, rule, out=out_static)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            olmoe.forward(x_static, rule, rule, out=out_static)
+        for b in (121, 122):
+            x = olmoe.tokens(B, synth.token_seed(olmoe.shape, b))
+            x_static.copy_(x)
+            graph.replay()
+            ref = torch.empty_like(x)
+            olmoe.forward(x, rule, rule, out=ref)
+            torch.cuda.synchronize()
+            got, want = out_static.float(), ref.float()
+            # same kernels on the same inputs; only the order of the fp32 reductions differs
+            scale = want.pow(2).mean().sqrt()
+            assert ((got - want).abs() <= 1e-2 * torch.maximum(want.abs(), scale)).all()
+        del graph
+    finally:
+        moe_set_dense_min_tokens(olmoe.h, DEFAULT_DENSE_MIN)
