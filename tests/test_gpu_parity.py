@@ -294,3 +294,41 @@ def test_forward_replays_in_a_cuda_graph(olmoe, B, dense_min):
         del graph
     finally:
         moe_set_dense_min_tokens(olmoe.h, DEFAULT_DENSE_MIN)
+
+
+# ---------------------------------------------------------------------------------------------
+# shapes off the register-fragment variants and at the configuration limits
+def _shape(name, H, E, k, I, S=0, Ish=0, **kw):
+    return synth.configs.LayerShape(name, H, E, k, I, n_shared=S, inter_shared=Ish, **kw)
+
+
+@pytest.mark.parametrize("B", [4, 33])
+def test_generic_variant_hidden_1024(B):
+    # H = 1024 has no register-fragment variant: token tiles go through shared memory
+    shape = _shape("h1024", 1024, 32, 4, 256, S=1, Ish=384)
+    dl = DeviceLayer(shape, max_tokens=64)
+    try:
+        _run(dl, B, ("topk", 0.5), ("topk", 0.9), batch_index=B)
+    finally:
+        dl.close()
+
+
+def test_wide_routing_many_experts():
+    # E = 256, top-16 (the top-k limit), H = 192 (generic variant), I = 96
+    shape = _shape("wide", 192, 256, 16, 96)
+    dl = DeviceLayer(shape, max_tokens=40)
+    try:
+        _run(dl, 40, ("topk", 0.75), batch_index=3)
+        _run(dl, 1, ("topk", 0.0), batch_index=4)
+    finally:
+        dl.close()
+
+
+def test_largest_intermediate():
+    # I = 16384 (the limit): 512 keys per select thread, 512-word union rows
+    shape = _shape("i16k", 256, 4, 2, 16384, S=1, Ish=16384)
+    dl = DeviceLayer(shape, max_tokens=8)
+    try:
+        _run(dl, 8, ("topk", 0.9), ("topk", 0.5), batch_index=1)
+    finally:
+        dl.close()
