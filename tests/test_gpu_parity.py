@@ -309,6 +309,10 @@ def test_generic_variant_hidden_1024(B):
     dl = DeviceLayer(shape, max_tokens=64)
     try:
         _run(dl, B, ("topk", 0.5), ("topk", 0.9), batch_index=B)
+        # the same shape on the tensor-core path: ragged token tiles, threshold mode for the
+        # shared expert
+        moe_set_dense_min_tokens(dl.h, 1)
+        _run(dl, B, ("topk", 0.9), ("threshold", 0.05), batch_index=B + 1)
     finally:
         dl.close()
 
