@@ -10,7 +10,11 @@
  *
  * Conventions shared by every entry point
  *   - Plain C types only.  `stream` is a cudaStream_t passed as void* (NULL = legacy default
- *     stream).  Device pointers are CUDA global-memory addresses of the current device.
+ *     stream).  Device pointers are CUDA global-memory addresses.
+ *   - A handle belongs to the device that was current at moe_create.  Every call on it makes
+ *     that device current for the call's duration and then restores the caller's device.
+ *     Its buffers and `stream` must belong to that device.  Calls without a handle, such as
+ *     moe_route_noalloc, run on the current device.
  *   - The caller owns every buffer it passes.  The handle owns its workspace (allocated once
  *     by moe_create, sized for cfg.max_tokens) and never allocates afterwards, so moe_forward
  *     makes no allocation and no host synchronisation and may be captured in a CUDA graph.

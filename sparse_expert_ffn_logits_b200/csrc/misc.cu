@@ -115,7 +115,8 @@ cudaError_t launch_pack_down(const void* w_down, void* packed_updown, int n, int
   dim3 grid((I + 31) / 32, (H + 31) / 32, n), block(32, 8);
   if (elt == 2)
     pack_down_kernel<__nv_bfloat16><<<grid, block, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(w_down), static_cast<__nv_bfloat16*>(packed_updown), I, H);
+        static_cast<const __nv_bfloat16*>(w_down), static_cast<__nv_bfloat16*>(packed_updown), I,
+        H);
   else
     pack_down_kernel<float><<<grid, block, 0, st>>>(static_cast<const float*>(w_down),
                                                     static_cast<float*>(packed_updown), I, H);

@@ -65,6 +65,27 @@ int auto_dense_min(const moe_config& c, int n_tokens, const moe_sparsity* sp) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Makes the handle's device current for one call and restores the caller's device after it,
+// so that a handle works whichever device the calling thread has selected.
+struct DeviceScope {
+  int prev = -1;
+  bool switched = false;
+  bool ok = true;
+  explicit DeviceScope(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) {
+      ok = false;
+      return;
+    }
+    if (prev != dev) {
+      ok = cudaSetDevice(dev) == cudaSuccess;
+      switched = ok;
+    }
+  }
+  ~DeviceScope() {
+    if (switched) cudaSetDevice(prev);
+  }
+};
+
 moe_status check_config(const moe_config* c) {
   if (!c) return MOE_ERR_INVALID_ARG;
   if (c->dtype != MOE_BF16 && c->dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
@@ -320,6 +341,8 @@ moe_status moe_pack_experts(moe_handle* h, int shared, const void* w_gate, const
   if (shared && h->cfg.n_shared == 0) return MOE_ERR_INVALID_ARG;
   if (n > (shared ? h->cfg.n_shared : h->cfg.n_routed)) return MOE_ERR_INVALID_ARG;
   if (n == 0) return MOE_OK;
+  DeviceScope dev(h->device);
+  if (!dev.ok) return MOE_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t H = h->cfg.hidden, I = shared ? h->cfg.inter_shared : h->cfg.inter, elt = h->elt;
   cudaError_t e = cudaSuccess;
@@ -328,7 +351,8 @@ moe_status moe_pack_experts(moe_handle* h, int shared, const void* w_gate, const
   if (e == cudaSuccess)
     e = cudaMemcpy2DAsync(packed_updown, 2 * H * elt, w_up, H * elt, H * elt, (size_t)n * I,
                           cudaMemcpyDeviceToDevice, st);
-  if (e == cudaSuccess) e = moe::launch_pack_down(w_down, packed_updown, n, (int)I, (int)H, (int)elt, st);
+  if (e == cudaSuccess)
+    e = moe::launch_pack_down(w_down, packed_updown, n, (int)I, (int)H, (int)elt, st);
   return cuda_status(e);
 }
 
@@ -340,6 +364,8 @@ moe_status moe_forward(moe_handle* h, const void* x, int n_tokens, const void* r
                                false);
   if (s != MOE_OK) return s;
   if (n_tokens == 0) return MOE_OK;
+  DeviceScope dev(h->device);
+  if (!dev.ok) return MOE_ERR_CUDA;
   return forward_impl(h, x, n_tokens, router, routed, shared, sp_routed, sp_shared, out,
                       static_cast<cudaStream_t>(stream));
 }
@@ -352,6 +378,8 @@ moe_status moe_forward_host(moe_handle* h, const void* x_host, int n_tokens, con
                                out_host, true);
   if (s != MOE_OK) return s;
   if (n_tokens == 0) return MOE_OK;
+  DeviceScope dev(h->device);
+  if (!dev.ok) return MOE_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t bytes = (size_t)n_tokens * h->cfg.hidden * h->elt;
   if (cudaMemcpyAsync(h->x_stage, x_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
@@ -367,6 +395,8 @@ moe_status moe_forward_host(moe_handle* h, const void* x_host, int n_tokens, con
 moe_status moe_debug_lists(moe_handle* h, int n_tokens, int* idx, float* w, float* logits,
                            int* cnt, int* lists, float* act, void* stream) {
   if (!h || n_tokens <= 0 || n_tokens != h->last_tokens) return MOE_ERR_INVALID_ARG;
+  DeviceScope dev(h->device);
+  if (!dev.ok) return MOE_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const moe_config& c = h->cfg;
   FwdParams p = h->base;
@@ -410,18 +440,19 @@ moe_status moe_read_trace(moe_handle* h, unsigned long long* host, size_t n) {
   if (!h || !host) return MOE_ERR_INVALID_ARG;
   const size_t cap = (size_t)moe::kTraceKernels * moe::kTraceCtas * moe::kTracePoints;
   if (n > cap) n = cap;
-  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  DeviceScope dev(h->device);
+  if (!dev.ok || cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
   if (cudaMemcpy(host, h->trace_buf, n * sizeof(unsigned long long), cudaMemcpyDeviceToHost) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
-  return cudaMemset(h->trace_buf, 0, n * sizeof(unsigned long long)) == cudaSuccess ? MOE_OK
-                                                                                      : MOE_ERR_CUDA;
+  return cuda_status(cudaMemset(h->trace_buf, 0, n * sizeof(unsigned long long)));
 }
 
 moe_status moe_get_error(moe_handle* h, int* device_code) {
   if (!h || !device_code) return MOE_ERR_INVALID_ARG;
   *device_code = 0;
-  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  DeviceScope dev(h->device);
+  if (!dev.ok || cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
   int v = 0;
   if (cudaMemcpy(&v, h->base.err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
     return MOE_ERR_CUDA;
@@ -433,6 +464,8 @@ moe_status moe_get_error(moe_handle* h, int* device_code) {
 
 moe_status moe_debug_force_timeout(moe_handle* h, void* stream) {
   if (!h) return MOE_ERR_INVALID_ARG;
+  DeviceScope dev(h->device);
+  if (!dev.ok) return MOE_ERR_CUDA;
   return cuda_status(moe::launch_force_timeout(h->base, static_cast<cudaStream_t>(stream)));
 }
 
@@ -444,10 +477,15 @@ moe_status moe_set_dense_min_tokens(moe_handle* h, int min_tokens) {
 
 moe_status moe_destroy(moe_handle* h) {
   if (!h) return MOE_OK;
-  cudaError_t e = cudaDeviceSynchronize();
-  cudaError_t f = cudaFree(h->ws);
+  moe_status s = MOE_OK;
+  {
+    DeviceScope dev(h->device);
+    cudaError_t e = dev.ok ? cudaDeviceSynchronize() : cudaErrorInvalidDevice;
+    cudaError_t f = cudaFree(h->ws);
+    if (e != cudaSuccess || f != cudaSuccess) s = MOE_ERR_CUDA;
+  }
   delete h;
-  return (e == cudaSuccess && f == cudaSuccess) ? MOE_OK : MOE_ERR_CUDA;
+  return s;
 }
 
 const char* moe_status_string(moe_status s) {

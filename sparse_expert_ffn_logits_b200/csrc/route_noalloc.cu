@@ -37,7 +37,8 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) unsigned char g_route_scratch[kScratchBytes];
 
 std::mutex g_setup_mu;
-void* g_scratch_addr[kMaxDevices];  // device address of g_route_scratch per device; null = not set up
+// device address of g_route_scratch per device; null = not set up yet
+void* g_scratch_addr[kMaxDevices];
 
 // Once per device, with that device current: the scratch area's address and the router
 // kernels' shared-memory limit.  Returns the address, or null (with *err set) on failure.
