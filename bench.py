@@ -3,8 +3,10 @@
 One step = one layer call (router, gate, selection, sparse up/down, output cast) on one batch
 of synthetic decode tokens.  Default workload: the OLMoE-shaped bf16 layer (H2048, 64 experts,
 top-8, I1024) at 16 tokens and 90 % intra-expert sparsity; ``--sweep`` adds the batch x
-sparsity grid (1..256 tokens, s = 0 / 0.5 / 0.9).  L2 is flushed (a 2x-L2 buffer is written)
-before every timed step and the token batch rotates through a pool of 32.
+sparsity grid (1..256 tokens, s = 0 / 0.5 / 0.9).  L2 is flushed (a 2x-L2 buffer is written,
+then another is read) before every timed step and the token batch rotates through a pool of 32.
+The line also reports the same steps replayed from CUDA graphs (``graph``) and through the
+host-buffer call with its copies (``e2e``).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cuda|reference]
 
@@ -20,6 +22,7 @@ import statistics
 import subprocess
 import sys
 import tempfile
+import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -61,18 +64,56 @@ def peaks():
 
 # ---------------------------------------------------------------------------------------------
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    """SM clock and throttle reasons sampled during the timed region.
+
+    NVML is polled about every millisecond from a background thread (read-only queries; ctypes
+    releases the GIL, so the launch loop is not held up), which gives samples even when the
+    timed region lasts only milliseconds.  Without NVML, nvidia-smi samples every 200 ms."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, device_index):
-        self.dev = device_index
+    def __init__(self, device_id):
+        self.dev = device_id  # "GPU-<uuid>" or an index
         self.proc = None
         self.path = None
+        self.thread = None
+        self.samples = []
+
+    def _nvml_handle(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            if str(self.dev).startswith("GPU-"):
+                return pynvml, pynvml.nvmlDeviceGetHandleByUUID(str(self.dev))
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(int(self.dev))
+        except Exception:
+            return None, None
 
     def start(self):
+        nv, h = self._nvml_handle()
+        if h is not None:
+            bits = {n: getattr(nv, "nvmlClocksEventReason" + c)
+                    for n, c in zip(self.REASONS, ("HwSlowdown", "HwThermalSlowdown",
+                                                   "SwThermalSlowdown", "SwPowerCap"))}
+            self.stop_flag = threading.Event()
+
+            def poll():
+                while not self.stop_flag.is_set():
+                    try:
+                        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+                        rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.samples.append((sm, mx, [n for n, b in bits.items() if rs & b]))
+                    except Exception:
+                        break
+                    time.sleep(0.001)
+
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            return
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
@@ -84,6 +125,17 @@ class ClockSampler:
             self.proc = None
 
     def stop(self):
+        if self.thread is not None:
+            self.stop_flag.set()
+            self.thread.join(timeout=5)
+            rows = self.samples
+            if not rows:
+                return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"],
+                        "source": "nvml"}
+            return {"sm_mhz": statistics.median(r[0] for r in rows),
+                    "sm_max_mhz": max(r[1] for r in rows),
+                    "reasons": sorted({n for r in rows for n in r[2]}),
+                    "samples": len(rows), "source": "nvml"}
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -98,12 +150,12 @@ class ClockSampler:
                 rows.append(parts)
         os.unlink(self.path)
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"],
+                    "source": "nvidia-smi"}
+        reasons = sorted({n for r in rows for n, v in zip(self.REASONS, r[5:9]) if v == "Active"})
         return {"sm_mhz": statistics.median(int(r[1]) for r in rows),
                 "sm_max_mhz": max(int(r[2]) for r in rows), "reasons": reasons,
-                "samples": len(rows)}
+                "samples": len(rows), "source": "nvidia-smi"}
 
 
 # ---------------------------------------------------------------------------------------------
@@ -312,6 +364,36 @@ def run_cuda(args, rank, world, local_rank):
            "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes,
            "api": "moe_forward_host"}
 
+    # ---- the same steps replayed from CUDA graphs: one captured layer call per pooled batch
+    # (the five launches and their programmatic edges are recorded once, replayed per step)
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        dl.forward(xs[0], rule, rule, out=out)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graphs = []
+    for i in range(pool_n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            dl.forward(xs[i], rule, rule, out=out)
+        graphs.append(g)
+    for i in range(args.warmup):
+        graphs[i % pool_n].replay()
+    torch.cuda.synchronize()
+    g_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        g_ev[i][0].record()
+        graphs[i % pool_n].replay()
+        g_ev[i][1].record()
+    torch.cuda.synchronize()
+    g_ms = job_time_ms(sum(a.elapsed_time(b) for a, b in g_ev), world, dev)
+    graph = {"value": round(job_throughput(world, B, args.steps, g_ms), 1), "unit": UNIT,
+             "ms_per_step": round(g_ms / args.steps, 5), "graphs": pool_n}
+    del graphs
+
     # ---- sweep (rank 0, single GPU)
     sweep = []
     if sweep_on and rank == 0:
@@ -354,7 +436,7 @@ def run_cuda(args, rank, world, local_rank):
                        "l2": "flushed before every step: a 2x-L2 buffer written, then another "
                              "2x-L2 buffer read (clean lines, none of the layer's)",
                        "token_pool": pool_n, "parallelism": f"replicas x{world}"},
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "graph": graph,
             "gpu_launches": 5 * args.steps, "clocks": clock_info}
     if sweep:
         line["sweep"] = sweep
