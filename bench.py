@@ -159,6 +159,14 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------------------------
+def workload_config(shape, B, world, s):
+    """The workload keys of `config`, the same in both arms (each arm adds how it ran)."""
+    return {"workload": f"{shape.name}-shaped MoE layer", "hidden": shape.hidden,
+            "experts": shape.n_routed, "top_k": shape.top_k, "inter": shape.inter,
+            "shared": shape.n_shared, "batch_per_gpu": B, "global_batch": B * world,
+            "sparsity": s, "selection": "top-K per (token, expert)"}
+
+
 def algorithmic_bytes(shape, dbg, B):
     """Bytes the method must read per stage for one call (each touched expert's gate block
     once, each kept row of the per-expert union once), from the call's kept lists."""
@@ -429,13 +437,10 @@ def run_cuda(args, rank, world, local_rank):
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(total_ms / args.steps, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": shape.dtype, "data": "synthetic",
-            "config": {"workload": f"{shape.name}-shaped MoE layer", "hidden": shape.hidden,
-                       "experts": shape.n_routed, "top_k": shape.top_k, "inter": shape.inter,
-                       "shared": shape.n_shared, "batch_per_gpu": B, "global_batch": B * world,
-                       "sparsity": s, "selection": "top-K per (token, expert)",
-                       "l2": "flushed before every step: a 2x-L2 buffer written, then another "
-                             "2x-L2 buffer read (clean lines, none of the layer's)",
-                       "token_pool": pool_n, "parallelism": f"replicas x{world}"},
+            "config": dict(workload_config(shape, B, world, s),
+                           l2="flushed before every step: a 2x-L2 buffer written, then another "
+                              "2x-L2 buffer read (clean lines, none of the layer's)",
+                           token_pool=pool_n, parallelism=f"replicas x{world}"),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "graph": graph,
             "gpu_launches": 5 * args.steps, "clocks": clock_info}
     if sweep:
@@ -517,10 +522,8 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"{shape.name}-shaped MoE layer", "hidden": shape.hidden,
-                       "experts": shape.n_routed, "top_k": shape.top_k, "inter": shape.inter,
-                       "shared": shape.n_shared, "batch_per_gpu": B, "sparsity": args.sparsity,
-                       "parallelism": "host cores"},
+            "config": dict(workload_config(shape, B, args.gpus, args.sparsity),
+                           token_pool=len(x_all), parallelism="host cores"),
             "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": oracle.threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,

@@ -64,3 +64,13 @@ def test_union_form_with_shared_experts():
     assert got["rows"] == rows == 8
     assert got["updown"] == rows * 2 * H * elt
     assert got["select"] == 3 * (1 + 2) * 96 * 4
+
+
+def test_both_arms_describe_the_workload_with_the_same_keys():
+    b = _bench()
+    shape = LayerShape("olmoe", 2048, 64, 8, 1024)
+    one = b.workload_config(shape, 16, 1, 0.9)
+    four = b.workload_config(shape, 16, 4, 0.9)
+    assert one["global_batch"] == 16 and four["global_batch"] == 64
+    assert set(one) == {"workload", "hidden", "experts", "top_k", "inter", "shared",
+                        "batch_per_gpu", "global_batch", "sparsity", "selection"}
