@@ -33,6 +33,12 @@ MUTANTS = [
     ("softmax_all_as_topk", "if (L.route == 1) {\n    for (int e = 0; e < E; ++e) z +=",
      "if (L.route == 99) {\n    for (int e = 0; e < E; ++e) z +=", 0),
     ("weight_not_applied", "o[h] += wj * yj[h];", "o[h] += yj[h];", 0),
+    ("score_from_gate", "score[n] = fabs(a[n]);", "score[n] = fabs(g[n]);", 0),
+    ("calibration_score_from_gate", "scores[(size_t)job * In + n] = fabs(a[n]);",
+     "scores[(size_t)job * In + n] = fabs(g[n]);", 0),
+    ("router_transposed", "load(L.router, L.elt, (size_t)e * H + h)",
+     "load(L.router, L.elt, (size_t)h * E + e)", 0),
+    ("calibration_ceil", "(long long)floor(s * (double)N)", "(long long)ceil(s * (double)N)", 0),
 ]
 
 
