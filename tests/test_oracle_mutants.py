@@ -39,6 +39,8 @@ MUTANTS = [
     ("router_transposed", "load(L.router, L.elt, (size_t)e * H + h)",
      "load(L.router, L.elt, (size_t)h * E + e)", 0),
     ("calibration_ceil", "(long long)floor(s * (double)N)", "(long long)ceil(s * (double)N)", 0),
+    ("shared_uses_routed_sparsity", "      sel = shared;", "      sel = routed;", 0),
+    ("h_from_g_not_silu", "keep, a.data(), &y", "keep, g.data(), &y", 0),
 ]
 
 
