@@ -93,3 +93,30 @@ def test_status_strings(lib):
     for s in range(7):
         assert lib.moe_status_string(s)
     assert lib.moe_status_string(99) == b"unknown status"
+
+
+@pytest.mark.parametrize("kw,n,ptrs,status", [
+    (dict(), -1, (16, 16, 16, 16), moe.MOE_ERR_INVALID_ARG),        # negative count
+    (dict(), 257, (16, 16, 16, 16), moe.MOE_ERR_UNSUPPORTED),       # beyond the scratch area
+    (dict(), 0, (0, 0, 0, 0), moe.MOE_OK),                          # a no-op reads nothing
+    (dict(), 4, (0, 16, 16, 16), moe.MOE_ERR_INVALID_ARG),          # null x
+    (dict(), 4, (16, 0, 16, 16), moe.MOE_ERR_INVALID_ARG),          # null router
+    (dict(), 4, (16, 16, 0, 16), moe.MOE_ERR_INVALID_ARG),          # null topk_idx
+    (dict(), 4, (16, 16, 16, 0), moe.MOE_ERR_INVALID_ARG),          # null topk_w
+    (dict(), 4, (8, 16, 16, 16), moe.MOE_ERR_INVALID_ARG),          # x not 16-byte aligned
+    (dict(), 4, (16, 8, 16, 16), moe.MOE_ERR_INVALID_ARG),          # router not 16-byte aligned
+    (dict(), 4, (16, 16, 2, 16), moe.MOE_ERR_INVALID_ARG),          # topk_idx not 4-byte aligned
+    (dict(hidden=96), 4, (16, 16, 16, 16), moe.MOE_ERR_UNSUPPORTED),  # hidden not a multiple of 64
+    (dict(top_k=65), 4, (16, 16, 16, 16), moe.MOE_ERR_INVALID_ARG),  # top_k above n_routed
+    (dict(n_routed=600, top_k=8), 4, (16, 16, 16, 16), moe.MOE_ERR_UNSUPPORTED),
+])
+def test_route_noalloc_rejects_bad_arguments_before_the_device(lib, kw, n, ptrs, status):
+    """Every check of the routing-only call runs on the host, before the scratch area (and so
+    the device) is touched: these pointers are never dereferenced."""
+    x, router, idx, w = (ctypes.c_void_p(p) if p else None for p in ptrs)
+    assert lib.moe_route_noalloc(ctypes.byref(_cfg(**kw)), x, n, router, idx, w, None) == status
+
+
+def test_route_noalloc_rejects_null_config(lib):
+    p = ctypes.c_void_p(16)
+    assert lib.moe_route_noalloc(None, p, 4, p, p, p, None) == moe.MOE_ERR_INVALID_ARG
