@@ -58,13 +58,16 @@ def _bind(lib):
     lib.oracle_route_weights.argtypes = [ctypes.POINTER(_Layer), P, P, P]
     lib.oracle_topk.argtypes = [P, ctypes.c_int, ctypes.c_int, P]
     lib.oracle_gate.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P]
+    lib.oracle_gate_tokens.argtypes = [P, ctypes.c_int, P, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_int, P, ctypes.c_int]
     lib.oracle_select.argtypes = [P, ctypes.c_int, _Sel, P]
     lib.oracle_expert.argtypes = [P, P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P]
     lib.oracle_forward.argtypes = [ctypes.POINTER(_Layer), P, ctypes.c_int, _Sel, _Sel, P, P, P,
                                    P, P, P, P, P, P, ctypes.c_int]
     lib.oracle_calibrate.argtypes = [ctypes.POINTER(_Layer), P, ctypes.c_int, ctypes.c_int,
                                      ctypes.c_double, P, P, ctypes.c_int]
-    for f in ("oracle_route", "oracle_route_weights", "oracle_topk", "oracle_gate", "oracle_select",
+    for f in ("oracle_route", "oracle_route_weights", "oracle_topk", "oracle_gate",
+              "oracle_gate_tokens", "oracle_select",
               "oracle_expert", "oracle_forward", "oracle_calibrate"):
         getattr(lib, f).restype = ctypes.c_int
     return lib
@@ -215,6 +218,19 @@ def gate(x_t, wg, lib=None):
     g = np.zeros(I); a = np.zeros(I)
     _check(lib.oracle_gate(_ptr(x_t), _ptr(wg), _elt(wg), H, I, _ptr(g), _ptr(a)), "oracle_gate")
     return g, a
+
+
+def gate_tokens(xs, wg, nthreads=0, lib=None):
+    """a [T][I] = SiLU(W_g x_t) of one expert for the T tokens xs [T][H] (host threads)."""
+    lib = lib or load()
+    xs = np.ascontiguousarray(xs); wg = np.ascontiguousarray(wg)
+    assert _elt(xs) == _elt(wg)
+    I, H = wg.shape
+    T = xs.shape[0]
+    a = np.zeros((T, I))
+    _check(lib.oracle_gate_tokens(_ptr(xs), T, _ptr(wg), _elt(wg), H, I, _ptr(a), int(nthreads)),
+           "oracle_gate_tokens")
+    return a
 
 
 def select(score, rule, lib=None):

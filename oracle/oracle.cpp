@@ -256,6 +256,23 @@ int oracle_gate(const void* x_t, const void* wg, int elt, int H, int I, double* 
   return ORACLE_OK;
 }
 
+/* Dense gate of one expert for T tokens: a [T][I] = SiLU(W_g x_t), the same loop as
+ * oracle_gate, with the (token, block of 64 neurons) jobs spread over the host threads. */
+int oracle_gate_tokens(const void* x, int T, const void* wg, int elt, int H, int I, double* a,
+                       int nthreads) {
+  if (!x || !wg || !a || T < 0 || H <= 0 || I <= 0 || (elt != 2 && elt != 4))
+    return ORACLE_BAD_ARG;
+  const int nb = (I + 63) / 64;
+  parallel_for(T * nb, nthreads, [&](int job) {
+    const int t = job / nb, n0 = (job % nb) * 64, n1 = std::min(I, n0 + 64);
+    const void* xt = static_cast<const char*>(x) + (size_t)t * H * elt;
+    const void* rows = static_cast<const char*>(wg) + (size_t)n0 * H * elt;
+    std::vector<double> g(n1 - n0);
+    gate_pair(xt, rows, elt, H, n1 - n0, g.data(), a + (size_t)t * I + n0);
+  });
+  return ORACLE_OK;
+}
+
 /* Kept-neuron mask keep [I] (0/1) from scores [I]. */
 int oracle_select(const double* score, int I, oracle_sel sel, unsigned char* keep) {
   if (!score || !keep || I <= 0 || !sel_ok(sel)) return ORACLE_BAD_ARG;

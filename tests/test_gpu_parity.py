@@ -184,7 +184,7 @@ def test_dsv2l(dsv2l, B, s, s_sh):
 # ---------------------------------------------------------------------------------------------
 @pytest.fixture(scope="module")
 def gptoss():
-    dl = DeviceLayer(synth.GPTOSS, max_tokens=64)
+    dl = DeviceLayer(synth.GPTOSS, max_tokens=256)
     yield dl
     dl.close()
 
@@ -194,6 +194,12 @@ def gptoss():
 def test_gptoss(gptoss, B, s):
     tokens = None if B <= 8 else np.arange(0, B, 4)
     _run(gptoss, B, ("topk", s), batch_index=B, tokens=tokens)
+
+
+def test_gptoss_large_batch(gptoss):
+    # 128 experts x 256 tokens of logits exceed the single-cluster router's shared memory: the
+    # multi-CTA router with its tickets; every token's routing and kept sets are checked
+    _run(gptoss, 256, ("topk", 0.5), batch_index=250, tokens=np.arange(0, 256, 16))
 
 
 @pytest.mark.parametrize("s", [0.5, 0.9])
@@ -221,13 +227,30 @@ def test_llama4(llama4, B, s):
     _run(llama4, B, ("topk", s), ("topk", s), batch_index=B)
 
 
-def test_llama4_large_batch(llama4):
-    shared = parity.host_shared(llama4.shape)
+@pytest.fixture(scope="module")
+def llama4_shared():
+    return parity.host_shared(synth.LLAMA4)
+
+
+def test_llama4_large_batch(llama4, llama4_shared):
+    # routing and kept sets of every token; the output of sampled tokens
     cache = {}
     _run(llama4, 256, ("topk", 0.9), ("topk", 0.9), batch_index=99, tokens=[0, 77, 255],
-         shared_weights=shared, expert_cache=cache)
+         shared_weights=llama4_shared, expert_cache=cache)
     _run(llama4, 64, ("topk", 0.5), ("topk", 0.5), batch_index=98, tokens=[1, 33, 63],
-         shared_weights=shared, expert_cache=cache)
+         shared_weights=llama4_shared, expert_cache=cache)
+
+
+@pytest.mark.parametrize("B,s", [(64, 0.9), (256, 0.5)])
+def test_llama4_shared_expert_dense(llama4, llama4_shared, B, s):
+    """Only the shared expert (B tokens) reaches 64 tokens: it takes the tensor-core path at
+    H = 5120, I = 8192, while the routed experts (about B / 128 tokens each) stay sparse."""
+    moe_set_dense_min_tokens(llama4.h, 64)
+    try:
+        _run(llama4, B, ("topk", s), ("topk", s), batch_index=200 + B, tokens=[0, B // 2, B - 1],
+             shared_weights=llama4_shared)
+    finally:
+        moe_set_dense_min_tokens(llama4.h, DEFAULT_DENSE_MIN)
 
 
 # ---------------------------------------------------------------------------------------------
