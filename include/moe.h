@@ -212,11 +212,12 @@ moe_status moe_destroy(moe_handle* h);
  *                                 the lower expert index
  *   topk_w    [n_tokens][top_k]   device fp32, written: the routing weights of cfg->route
  *   stream    cudaStream_t, or NULL for the default stream; the call is asynchronous
- * It runs on a 2 MiB scratch area that the library holds per device.  n_tokens <= 256;
- * n_tokens > 256 is UNSUPPORTED, n_tokens < 0 INVALID_ARG, n_tokens = 0 a no-op.  The first call
- * on a device sets the scratch area up (it may load the module), so make it before any stream
- * capture.  Calls that overlap in time on one device share the scratch area and race: serialise
- * them.  A NaN logit ranks lowest; no device error word is reported. */
+ * It runs on a 2 MiB scratch area that the library holds on every device that loads it, until
+ * the process exits.  n_tokens <= 256; n_tokens > 256 is UNSUPPORTED, n_tokens < 0 INVALID_ARG,
+ * n_tokens = 0 a no-op.  The first call in a device's CUDA context (the first call on the device,
+ * and the first after a device reset) sets the scratch area up (it may load the module), so make
+ * it before any stream capture.  Calls that overlap in time on one device share the scratch area
+ * and race: serialise them.  A NaN logit ranks lowest; no device error word is reported. */
 moe_status moe_route_noalloc(const moe_config* cfg, const void* x, int n_tokens,
                              const void* router, int* topk_idx, float* topk_w, void* stream);
 

@@ -60,6 +60,7 @@ struct FwdParams {
   int H, E, k, S, I, Ish, B, Imax;
   int Bmax;         // max_tokens of the handle
   int hsplit;       // router slices of H
+  int router_cluster;  // CTAs of the single-cluster router on this device (0: multi-CTA only)
   int route;
   int sel_mode[2];  // [0] routed, [1] shared: 0 top-K, 1 threshold
   int sel_K[2];

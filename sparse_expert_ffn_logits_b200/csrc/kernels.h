@@ -3,6 +3,8 @@
 
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "tma.cuh"
 
@@ -16,7 +18,18 @@ struct LaunchShape {
   Ring ring_gate;     // copy ring of the bf16 gate kernel
   Ring ring_ud;       // copy ring of the bf16 up/down kernel
   int variant;        // register-fragment ring variant (0: generic token tiles in smem)
+  int router_cluster; // CTAs of the single-cluster router (0: only the multi-CTA router)
 };
+
+constexpr int kMaxDevices = 64;
+
+// Identity of the calling thread's current CUDA context, unique for the life of the process
+// (0 if it cannot be read).  A device reset ends a context; the next one has another identity.
+unsigned long long current_context_id();
+
+// Held while kernels are configured (function attributes, per-context discoveries), so that
+// handles created and routing set up from several threads do not interleave.
+std::mutex& setup_mutex();
 
 // dtype: 0 bf16, 1 fp32.  Each launcher returns the launch's cudaError_t.
 cudaError_t launch_router(const FwdParams& p, int dtype, cudaStream_t st);
@@ -34,8 +47,10 @@ cudaError_t configure_dense(int budget);
 cudaError_t launch_finalize(const FwdParams& p, int dtype, const LaunchShape& ls, cudaStream_t st,
                             bool pdl);
 
-// Set-up (called once per handle): shared-memory limits and persistent grid sizes.
+// Set-up (called once per handle, under setup_mutex): shared-memory limits and persistent grid
+// sizes.
 cudaError_t configure_kernels(int dtype, int imax, int max_E, int max_B, int H, LaunchShape* ls);
+cudaError_t configure_router(int budget, int* cluster_out);
 size_t router_smem_bytes(int E, int B);
 size_t select_smem_bytes(int imax);
 

@@ -1,10 +1,11 @@
 // misc.cu - output cast, weight packing, debug export and per-handle kernel configuration.
+#include <cuda.h>
+
 #include "kernels.h"
 #include "tma.cuh"
 
 namespace moe {
 
-cudaError_t configure_router(int budget);
 cudaError_t configure_select(int imax, int budget, int* occupancy);
 cudaError_t configure_gate(int dtype, int H, int smem_budget, LaunchShape* ls);
 cudaError_t configure_updown(int dtype, int H, int smem_budget, LaunchShape* ls);
@@ -152,6 +153,35 @@ cudaError_t launch_debug_gather(const FwdParams& p, int n_tokens, int* cnt, int*
   return cudaGetLastError();
 }
 
+std::mutex& setup_mutex() {
+  static std::mutex mu;
+  return mu;
+}
+
+unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(f);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(f);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
 cudaError_t configure_kernels(int dtype, int imax, int max_E, int max_B, int H, LaunchShape* ls) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -161,7 +191,7 @@ cudaError_t configure_kernels(int dtype, int imax, int max_E, int max_B, int H, 
   int budget = 0;
   e = cudaDeviceGetAttribute(&budget, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (e != cudaSuccess) return e;
-  e = configure_router(budget);
+  e = configure_router(budget, &ls->router_cluster);
   if (e != cudaSuccess) return e;
   int occ_sel = 0;
   e = configure_select(imax, budget, &occ_sel);

@@ -198,6 +198,7 @@ moe_status forward_impl(moe_handle* h, const void* x, int n_tokens, const void* 
   p.Imax = h->imax;
   p.Bmax = c.max_tokens;
   p.hsplit = moe::router_hsplit(c.n_routed, n_tokens, c.hidden);
+  p.router_cluster = h->ls.router_cluster;
   p.route = (int)c.route;
   p.sel_mode[0] = sp_routed->mode == MOE_SEL_THRESHOLD ? 1 : 0;
   p.sel_K[0] = keep_count(c.inter, sp_routed->sparsity);
@@ -298,8 +299,12 @@ moe_status moe_create(const moe_config* cfg, moe_handle** out) {
     delete h;
     return MOE_ERR_CUDA;
   }
-  cudaError_t e = moe::configure_kernels(cfg->dtype == MOE_BF16 ? 0 : 1, h->imax, cfg->n_routed,
-                                         cfg->max_tokens, cfg->hidden, &h->ls);
+  cudaError_t e;
+  {
+    std::lock_guard<std::mutex> lock(moe::setup_mutex());
+    e = moe::configure_kernels(cfg->dtype == MOE_BF16 ? 0 : 1, h->imax, cfg->n_routed,
+                               cfg->max_tokens, cfg->hidden, &h->ls);
+  }
   if (e != cudaSuccess) {
     delete h;
     return MOE_ERR_CUDA;

@@ -11,11 +11,13 @@
 // For them this entry point runs the router kernel of the layer (logit tiles, top-k, grouping)
 // on a fixed scratch area compiled into the library, instead of a handle's workspace.
 //
-// The scratch area is one static device array per device.  The first call on a device looks up
-// its address (cudaGetSymbolAddress, which may load the module) and sets the router kernels'
-// shared-memory limit.  That first call should therefore come before any stream capture.  Every
-// later call only clears the zero-at-start words and launches.  Calls that overlap in time on one
-// device, from two streams or two threads, share the scratch area and race: the caller
+// The scratch area is one static device array, which every device that loads the library
+// holds until the process exits.  The first call in a device's CUDA context looks up the array's
+// address there (cudaGetSymbolAddress, which may load the module) and sets the router kernels'
+// limits; that first call should therefore come before any stream capture.  A later call checks
+// that the context is still the one set up (a device reset ends a context; the call after it
+// sets up again), clears the zero-at-start words and launches.  Calls that overlap in time on
+// one device, from two streams or two threads, share the scratch area and race: the caller
 // serialises them.
 #include <climits>
 #include <mutex>
@@ -23,46 +25,57 @@
 #include "../../include/moe.h"
 #include "kernels.h"
 
-namespace moe {
-cudaError_t configure_router(int budget);
-}
-
 namespace {
 
 constexpr size_t kScratchBytes = (size_t)2 << 20;  // 2 MiB: room for 256 tokens x 512 experts
 constexpr int kNoAllocMaxTokens = 256;
-constexpr int kMaxDevices = 64;
 
 // The scratch area (zero at module load; the zero-at-start words are cleared again by every call).
 static __device__ __align__(256) unsigned char g_route_scratch[kScratchBytes];
 
-std::mutex g_setup_mu;
-// device address of g_route_scratch per device; null = not set up yet
-void* g_scratch_addr[kMaxDevices];
+// per device: the context that was set up, the scratch area's address there and the width of
+// the single-cluster router (ctx 0 = not set up yet)
+struct DeviceSetup {
+  unsigned long long ctx;
+  void* scratch;
+  int router_cluster;
+};
+DeviceSetup g_setup[moe::kMaxDevices];
 
-// Once per device, with that device current: the scratch area's address and the router
-// kernels' shared-memory limit.  Returns the address, or null (with *err set) on failure.
-void* scratch_for_current_device(cudaError_t* err) {
+// The scratch area's address and the router's cluster width for the current device, set up
+// once per device context with that device current.  Returns false (with *err set) on failure.
+bool setup_current_device(void** scratch, int* cluster, cudaError_t* err) {
   int dev = 0;
   *err = cudaGetDevice(&dev);
-  if (*err != cudaSuccess) return nullptr;
-  if (dev < 0 || dev >= kMaxDevices) {
+  if (*err != cudaSuccess) return false;
+  if (dev < 0 || dev >= moe::kMaxDevices) {
     *err = cudaErrorInvalidDevice;
-    return nullptr;
+    return false;
   }
-  std::lock_guard<std::mutex> lock(g_setup_mu);
-  if (!g_scratch_addr[dev]) {
+  std::lock_guard<std::mutex> lock(moe::setup_mutex());
+  // the context identity is read after the first runtime call, so the context exists
+  const unsigned long long ctx = moe::current_context_id();
+  DeviceSetup& d = g_setup[dev];
+  if (ctx == 0 || d.ctx != ctx) {
     void* ptr = nullptr;
     *err = cudaGetSymbolAddress(&ptr, g_route_scratch);
-    if (*err != cudaSuccess || !ptr) return nullptr;
+    if (*err != cudaSuccess || !ptr) {
+      if (*err == cudaSuccess) *err = cudaErrorInvalidSymbol;
+      return false;
+    }
     int budget = 0;
     *err = cudaDeviceGetAttribute(&budget, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    if (*err != cudaSuccess) return nullptr;
-    *err = moe::configure_router(budget);
-    if (*err != cudaSuccess) return nullptr;
-    g_scratch_addr[dev] = ptr;
+    if (*err != cudaSuccess) return false;
+    int c = 0;
+    *err = moe::configure_router(budget, &c);
+    if (*err != cudaSuccess) return false;
+    d.scratch = ptr;
+    d.router_cluster = c;
+    d.ctx = ctx;  // 0 when the identity cannot be read: set up again on every call
   }
-  return g_scratch_addr[dev];
+  *scratch = d.scratch;
+  *cluster = d.router_cluster;
+  return true;
 }
 
 size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
@@ -116,8 +129,10 @@ extern "C" moe_status moe_route_noalloc(const moe_config* cfg, const void* x, in
   if (off > kScratchBytes) return MOE_ERR_UNSUPPORTED;
 
   cudaError_t ce = cudaSuccess;
-  char* base = static_cast<char*>(scratch_for_current_device(&ce));
-  if (!base) return MOE_ERR_CUDA;
+  void* scratch = nullptr;
+  int cluster = 0;
+  if (!setup_current_device(&scratch, &cluster, &ce)) return MOE_ERR_CUDA;
+  char* base = static_cast<char*>(scratch);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(base + o_zero, 0, zero_bytes, st) != cudaSuccess) return MOE_ERR_CUDA;
 
@@ -132,6 +147,7 @@ extern "C" moe_status moe_route_noalloc(const moe_config* cfg, const void* x, in
   p.Imax = moe::kTileRows;
   p.Bmax = B;
   p.hsplit = hsplit;
+  p.router_cluster = cluster;
   p.route = (int)cfg->route;
   p.dense_min = INT_MAX;  // only the grouping's item counts read it; no later kernel runs
   p.x = x;

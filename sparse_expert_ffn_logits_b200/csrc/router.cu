@@ -433,8 +433,6 @@ __global__ void __launch_bounds__(kThreads) router_cluster_kernel(FwdParams p) {
   }
 }
 
-int g_router_cluster = 0;  // CTAs of the single-cluster router (0: not available)
-
 }  // namespace
 
 size_t router_smem_bytes(int E, int B) {
@@ -464,20 +462,20 @@ cudaError_t launch_router_t(const FwdParams& p, dim3 grid, size_t smem, cudaStre
 }
 
 // The single-cluster router holds the batch's partial logits in each CTA's shared memory.
-bool router_uses_cluster(int E, int B) {
-  return g_router_cluster > 0 && (size_t)E * B * 4 <= kRouterClusterPartBytes;
+bool router_uses_cluster(int cluster, int E, int B) {
+  return cluster > 0 && (size_t)E * B * 4 <= kRouterClusterPartBytes;
 }
 
 template <typename T, int PER>
 cudaError_t launch_router_cluster_t(const FwdParams& p, size_t smem, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(g_router_cluster);
+  cfg.gridDim = dim3(p.router_cluster);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = g_router_cluster;
+  attr[0].val.clusterDim.x = p.router_cluster;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
@@ -497,7 +495,7 @@ cudaError_t launch_router_cluster(const FwdParams& p, cudaStream_t st) {
 }
 
 cudaError_t launch_router(const FwdParams& p, int dtype, cudaStream_t st) {
-  if (router_uses_cluster(p.E, p.B))
+  if (router_uses_cluster(p.router_cluster, p.E, p.B))
     return dtype == 0 ? launch_router_cluster<__nv_bfloat16>(p, st)
                       : launch_router_cluster<float>(p, st);
   dim3 grid(((p.E + kTileRows - 1) / kTileRows) * p.hsplit, (p.B + kTileTok - 1) / kTileTok);
@@ -533,40 +531,59 @@ cudaError_t configure_router_cluster_t(int budget, bool wide) {
   return e;
 }
 
-cudaError_t configure_router(int budget) {
+// Shared-memory limits of every router kernel and, for the single-cluster router, the widest
+// cluster the device accepts (16 CTAs where allowed, else 8; 0: only the multi-CTA router).
+// Function attributes belong to the current device's context, so this runs for every handle
+// and every context (the caller holds the set-up lock); the width found is kept per context.
+cudaError_t configure_router(int budget, int* cluster_out) {
   cudaError_t e = configure_router_t<__nv_bfloat16>(budget);
   if (e != cudaSuccess) return e;
   e = configure_router_t<float>(budget);
   if (e != cudaSuccess) return e;
-  // single-cluster router: 16 CTAs where the device takes a cluster that wide, else 8
-  if (g_router_cluster == 0) {
-    int c = 0;
-    for (int want : {16, 8}) {
-      if (configure_router_cluster_t<__nv_bfloat16>(budget, want > 8) != cudaSuccess ||
-          configure_router_cluster_t<float>(budget, want > 8) != cudaSuccess)
-        continue;
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(want);
-      cfg.blockDim = dim3(kThreads);
-      cfg.dynamicSmemBytes = kRouterClusterPartBytes;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = want;
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, router_cluster_kernel<__nv_bfloat16, 16>, &cfg) ==
-              cudaSuccess &&
-          n > 0) {
-        c = want;
-        break;
-      }
-    }
-    cudaGetLastError();  // a refused cluster width is not an error of this call
-    g_router_cluster = c;
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static unsigned long long known_ctx[kMaxDevices];
+  static int known_width[kMaxDevices];
+  const unsigned long long ctx = current_context_id();
+  if (dev >= 0 && dev < kMaxDevices && ctx != 0 && known_ctx[dev] == ctx) {
+    const int c = known_width[dev];
+    if (c > 0 && (configure_router_cluster_t<__nv_bfloat16>(budget, c > 8) != cudaSuccess ||
+                  configure_router_cluster_t<float>(budget, c > 8) != cudaSuccess))
+      return cudaErrorInvalidConfiguration;
+    *cluster_out = c;
+    return cudaSuccess;
   }
+  int c = 0;
+  for (int want : {16, 8}) {
+    if (configure_router_cluster_t<__nv_bfloat16>(budget, want > 8) != cudaSuccess ||
+        configure_router_cluster_t<float>(budget, want > 8) != cudaSuccess)
+      continue;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(want);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kRouterClusterPartBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = want;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, router_cluster_kernel<__nv_bfloat16, 16>, &cfg) ==
+            cudaSuccess &&
+        n > 0) {
+      c = want;
+      break;
+    }
+  }
+  cudaGetLastError();  // a refused cluster width is not an error of this call
+  if (dev >= 0 && dev < kMaxDevices && ctx != 0) {
+    known_ctx[dev] = ctx;
+    known_width[dev] = c;
+  }
+  *cluster_out = c;
   return cudaSuccess;
 }
 

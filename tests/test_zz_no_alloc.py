@@ -36,14 +36,19 @@ def test_rejects_before_touching_the_device():
         assert e.value.status == status
 
 
+# 512 experts x 100 tokens of logits exceed the single-cluster router's shared memory, so this
+# shape takes the multi-CTA router, whose tickets start at zero on every call
+WIDE = synth.configs.LayerShape("wide-router", 256, 512, 8, 64)
+
+
 @pytest.mark.gpu
-@pytest.mark.parametrize("shape", [synth.OLMOE, synth.TINY], ids=lambda s: s.name)
-def test_matches_forward_routing_on_two_calls_in_a_row(shape):
-    dl = DeviceLayer(shape, max_tokens=64)
+@pytest.mark.parametrize("shape,sizes", [(synth.OLMOE, (16, 64)), (synth.TINY, (16, 64)),
+                                         (WIDE, (100, 96))], ids=lambda v: getattr(v, "name", ""))
+def test_matches_forward_routing_on_two_calls_in_a_row(shape, sizes):
+    dl = DeviceLayer(shape, max_tokens=max(sizes))
     try:
-        cfg = _cfg(shape)
-        batches = [(16, dl.tokens(16, synth.token_seed(shape, 3))),
-                   (64, dl.tokens(64, synth.token_seed(shape, 4)))]
+        cfg = _cfg(shape, max_tokens=max(sizes))
+        batches = [(B, dl.tokens(B, synth.token_seed(shape, 3 + i))) for i, B in enumerate(sizes)]
         want = []
         for B, x in batches:
             out = torch.empty_like(x)
