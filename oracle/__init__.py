@@ -56,6 +56,10 @@ def _bind(lib):
     lib.oracle_threads.restype = ctypes.c_int
     lib.oracle_route.argtypes = [ctypes.POINTER(_Layer), P, ctypes.c_int, P, P, P]
     lib.oracle_route_weights.argtypes = [ctypes.POINTER(_Layer), P, P, P]
+    lib.oracle_route_biased.argtypes = [ctypes.POINTER(_Layer), P, ctypes.c_int, P, P, P, P]
+    lib.oracle_roster_bias.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_double, P]
+    lib.oracle_roster_update.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int]
     lib.oracle_topk.argtypes = [P, ctypes.c_int, ctypes.c_int, P]
     lib.oracle_gate.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P]
     lib.oracle_gate_tokens.argtypes = [P, ctypes.c_int, P, ctypes.c_int, ctypes.c_int,
@@ -66,7 +70,8 @@ def _bind(lib):
                                    P, P, P, P, P, P, ctypes.c_int]
     lib.oracle_calibrate.argtypes = [ctypes.POINTER(_Layer), P, ctypes.c_int, ctypes.c_int,
                                      ctypes.c_double, P, P, ctypes.c_int]
-    for f in ("oracle_route", "oracle_route_weights", "oracle_topk", "oracle_gate",
+    for f in ("oracle_route", "oracle_route_biased", "oracle_roster_bias", "oracle_roster_update",
+              "oracle_route_weights", "oracle_topk", "oracle_gate",
               "oracle_gate_tokens", "oracle_select",
               "oracle_expert", "oracle_forward", "oracle_calibrate"):
         getattr(lib, f).restype = ctypes.c_int
@@ -154,6 +159,19 @@ class Layer:
                                      _ptr(w)), "oracle_route")
         return logits, idx, w
 
+    def route_biased(self, x, bias):
+        """Routing with an additive selection bias [B][E] (None: no bias): the top-k of
+        logits + bias, the weights from the unbiased logits.  Returns (logits, idx, w)."""
+        x = np.ascontiguousarray(x)
+        B, E, k = x.shape[0], self.shape.n_routed, self.shape.top_k
+        b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float64)
+        assert b is None or b.shape == (B, E)
+        logits = np.zeros((B, E)); idx = np.zeros((B, k), np.int32); w = np.zeros((B, k))
+        _check(self.lib.oracle_route_biased(ctypes.byref(self.c), _ptr(x), B, _ptr(b),
+                                            _ptr(logits), _ptr(idx), _ptr(w)),
+               "oracle_route_biased")
+        return logits, idx, w
+
     def route_weights(self, logits_row, idx_row):
         lg = np.ascontiguousarray(logits_row, dtype=np.float64)
         ix = np.ascontiguousarray(idx_row, dtype=np.int32)
@@ -218,6 +236,29 @@ def gate(x_t, wg, lib=None):
     g = np.zeros(I); a = np.zeros(I)
     _check(lib.oracle_gate(_ptr(x_t), _ptr(wg), _elt(wg), H, I, _ptr(g), _ptr(a)), "oracle_gate")
     return g, a
+
+
+def roster_bias(counts, pinned, m, delta, lib=None):
+    """Roster bias [B][E] (float64) from the selection counts [B][E] and pinned flags [B]."""
+    lib = lib or load()
+    c = np.ascontiguousarray(counts, dtype=np.int32)
+    pn = np.ascontiguousarray(pinned, dtype=np.int32)
+    B, E = c.shape
+    b = np.zeros((B, E))
+    _check(lib.oracle_roster_bias(_ptr(c), _ptr(pn), B, E, int(m), float(delta), _ptr(b)),
+           "oracle_roster_bias")
+    return b
+
+
+def roster_update(counts, idx, lib=None):
+    """counts[t][idx[t][j]] += 1, in place (counts: int32 [B][E], idx [B][k])."""
+    lib = lib or load()
+    assert counts.dtype == np.int32 and counts.flags.c_contiguous
+    ix = np.ascontiguousarray(idx, dtype=np.int32)
+    B, E = counts.shape
+    _check(lib.oracle_roster_update(_ptr(counts), _ptr(ix), B, E, ix.shape[1]),
+           "oracle_roster_update")
+    return counts
 
 
 def gate_tokens(xs, wg, nthreads=0, lib=None):

@@ -25,6 +25,14 @@
  *   layer output           out_t = sum_{e in topk(t)} w_{t,e} y_{t,e} + sum_sh y_{t,sh}
  *                          y = sum_{n in A} SiLU(g_n) (W_up[n] . x) W_down[:, n]
  *
+ * Optional roster routing ("Predatory MoE", technical summary, Methodology 2, the roster rule):
+ * each sequence counts how often each expert of the layer was selected; its roster is the m
+ * most-used experts (equal counts: lower expert index); while fewer than m distinct experts
+ * have been used there is no bias (exploration), afterwards roster members get +delta and the
+ * others -delta (barrier); a pinned sequence selects among its roster only (-inf for the
+ * others).  Readings: the bias enters the top-k choice only, the routing weights stay those of
+ * the unbiased logits; one decode token per sequence; the caller decides when to pin.
+ *
  * Inputs are passed exactly as stored for the device: bf16 bit patterns (elt = 2) or binary32
  * (elt = 4), widened exactly to double.
  */
@@ -217,6 +225,66 @@ int oracle_keep_count(int I, double s) { return keep_count(I, s); }
 int oracle_threads(void) {
   int hw = (int)std::thread::hardware_concurrency();
   return hw > 0 ? hw : 1;
+}
+
+/* Roster bias of B sequences: counts [B][E] selections so far, pinned [B] (0 / 1), budget m
+ * (1 <= m <= E), delta >= 0  ->  bias [B][E]. */
+int oracle_roster_bias(const int* counts, const int* pinned, int B, int E, int m, double delta,
+                       double* bias) {
+  if (!counts || !pinned || !bias || B < 0 || E <= 0 || m < 1 || m > E || !(delta >= 0.0))
+    return ORACLE_BAD_ARG;
+  std::vector<int> order(E);
+  for (int t = 0; t < B; ++t) {
+    const int* c = counts + (size_t)t * E;
+    for (int e = 0; e < E; ++e) order[e] = e;
+    std::sort(order.begin(), order.end(), [&](int p, int q) {
+      if (c[p] != c[q]) return c[p] > c[q];
+      return p < q;
+    });
+    std::vector<unsigned char> member(E, 0);
+    for (int r = 0; r < m; ++r) member[order[r]] = 1;
+    int distinct = 0;
+    for (int e = 0; e < E; ++e) distinct += c[e] > 0;
+    double* b = bias + (size_t)t * E;
+    for (int e = 0; e < E; ++e) {
+      if (pinned[t]) b[e] = member[e] ? 0.0 : -INFINITY;
+      else if (distinct < m) b[e] = 0.0;
+      else b[e] = member[e] ? delta : -delta;
+    }
+  }
+  return ORACLE_OK;
+}
+
+/* counts[t][idx[t][j]] += 1 for the k experts each sequence's token selected. */
+int oracle_roster_update(int* counts, const int* idx, int B, int E, int k) {
+  if (!counts || !idx || B < 0 || E <= 0 || k <= 0) return ORACLE_BAD_ARG;
+  for (int t = 0; t < B; ++t)
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(size_t)t * k + j];
+      if (e < 0 || e >= E) return ORACLE_BAD_ARG;
+      counts[(size_t)t * E + e] += 1;
+    }
+  return ORACLE_OK;
+}
+
+/* Router with an additive selection bias [B][E] (nullable): the top-k of logits + bias by
+ * (value descending, expert index ascending); the weights of the chosen experts from the
+ * unbiased logits.  logits [B][E] (nullable) are the unbiased ones. */
+int oracle_route_biased(const oracle_layer* L, const void* x, int B, const double* bias,
+                        double* logits, int* idx, double* w) {
+  if (!L || !L->router || B < 0 || !x || !idx || !w || L->top_k <= 0 || L->top_k > L->n_routed)
+    return ORACLE_BAD_ARG;
+  const int E = L->n_routed, k = L->top_k;
+  std::vector<double> lg(E), sel(E);
+  for (int t = 0; t < B; ++t) {
+    const void* xt = static_cast<const char*>(x) + (size_t)t * L->hidden * L->elt;
+    router_logits(*L, xt, lg.data());
+    for (int e = 0; e < E; ++e) sel[e] = lg[e] + (bias ? bias[(size_t)t * E + e] : 0.0);
+    topk_experts(sel.data(), E, k, idx + (size_t)t * k);
+    route_weights(*L, lg.data(), idx + (size_t)t * k, w + (size_t)t * k);
+    if (logits) memcpy(logits + (size_t)t * E, lg.data(), sizeof(double) * E);
+  }
+  return ORACLE_OK;
 }
 
 /* Router for B tokens.  logits [B][E] (nullable), idx [B][k], w [B][k]. */

@@ -15,6 +15,10 @@ What pins what:
   layer output    s = 0 equals the textbook dense SwiGLU MoE (torch fp64); s > 0 equals the
                   dense layer with an explicit 0/1 mask built by a full stable sort
   invariants      expert relabelling, batch independence, W_up scaling, calibration quantile
+  roster routing  the roster by brute force over m-subsets of the counts; the biased top-k by
+                  brute force with scipy weights on the unbiased logits; simulated sequences:
+                  no bias while exploring, a pinned sequence never leaves its m experts, and
+                  the barrier shrinks the experts a sequence uses
 """
 import itertools
 import sys
@@ -275,9 +279,101 @@ def pin_calibration(lib):
         assert int((sc > sc[m - 1]).sum()) == N - m
 
 
+def pin_roster_bias(lib):
+    rng = np.random.default_rng(11)
+    for trial in range(80):
+        E = int(rng.integers(3, 8))
+        m = int(rng.integers(1, E + 1))
+        counts = rng.integers(0, 4, size=(1, E)).astype(np.int32)
+        if trial % 3 == 0:
+            counts[0, rng.integers(0, E)] += 5
+        pinned = int(trial % 4 == 1)
+        delta = float(rng.choice([0.0, 0.25, 3.0]))
+        b = oracle.roster_bias(counts, [pinned], m, delta, lib=lib)[0]
+        roster = _brute_topk(counts[0].astype(np.float64), m)  # lower index wins equal counts
+        distinct = int((counts[0] > 0).sum())
+        for e in range(E):
+            if pinned:
+                want = 0.0 if roster[e] else -np.inf
+            elif distinct < m:
+                want = 0.0
+            else:
+                want = delta if roster[e] else -delta
+            assert b[e] == want, (counts, m, pinned, delta, e, b)
+    c = np.zeros((2, 5), np.int32)
+    oracle.roster_update(c, np.array([[4, 1], [0, 4]]), lib=lib)
+    oracle.roster_update(c, np.array([[4, 2], [3, 0]]), lib=lib)
+    assert c.tolist() == [[0, 1, 1, 0, 2], [2, 0, 0, 1, 1]]
+
+
+def pin_route_biased(lib):
+    shape = small_shape(route="softmax_topk", n_routed=7, top_k=3, n_shared=0, inter_shared=0)
+    router = synth.host_tensor(shape, "router")
+    for route in ("softmax_topk", "softmax_all", "sigmoid"):
+        sh = shape.with_(route=route)
+        layer = oracle.Layer(sh, router, {}, lib=lib)
+        x = synth.host_tokens(sh, 12, 31)
+        lg_ref = f32(x).astype(np.float64) @ f32(router).astype(np.float64).T
+        # no bias is the plain router
+        l0, i0, w0 = layer.route(x)
+        l1, i1, w1 = layer.route_biased(x, None)
+        assert np.array_equal(i0, i1) and np.array_equal(w0, w1)
+        rng = np.random.default_rng(5)
+        bias = rng.choice([0.0, 0.02, -0.02, 0.5, -np.inf], size=(12, 7))
+        bias[:, :3] = rng.choice([0.0, 0.02, -0.02], size=(12, 3))  # >= k finite entries
+        lg, idx, w = layer.route_biased(x, bias)
+        assert _rel(lg, lg_ref) < 1e-12
+        for t in range(12):
+            v = lg_ref[t] + bias[t]
+            want = _brute_topk(np.where(np.isinf(v), -1e30, v), sh.top_k)  # exact sums
+            got = np.zeros(7, np.uint8)
+            got[idx[t]] = 1
+            assert np.array_equal(got, want), (route, t)
+            if route == "softmax_topk":
+                w_ref = scipy.special.softmax(lg_ref[t][idx[t]])
+            elif route == "softmax_all":
+                w_ref = scipy.special.softmax(lg_ref[t])[idx[t]]
+            else:
+                w_ref = scipy.special.expit(lg_ref[t][idx[t]])
+            assert _rel(w[t], w_ref) < 1e-12, (route, w[t], w_ref)
+
+
+def pin_roster_sequences(lib):
+    """Decode steps of 24 sequences with the roster rule, on the oracle's own routing."""
+    shape = small_shape(n_routed=16, top_k=2, n_shared=0, inter_shared=0)
+    router = synth.host_tensor(shape, "router")
+    layer = oracle.Layer(shape, router, {}, lib=lib)
+    S, steps, m, pin_at = 24, 40, 4, 8
+    used = {}
+    for delta in (0.0, 0.05):
+        counts = np.zeros((S, 16), np.int32)
+        seen_after_pin = [set() for _ in range(S)]
+        for step in range(steps):
+            x = synth.host_tokens(shape, S, 400 + step)
+            pinned = np.full(S, int(delta > 0 and step >= pin_at), np.int32)
+            b = oracle.roster_bias(counts, pinned, m, delta, lib=lib)
+            _, idx, _ = layer.route_biased(x, b)
+            _, idx0, _ = layer.route(x)
+            for t in range(S):
+                if int((counts[t] > 0).sum()) < m and not pinned[t]:
+                    # exploring: the choice is the router's own
+                    assert np.array_equal(idx[t], idx0[t])
+                if pinned[t]:
+                    # the roster (pinned by brute force in pin_roster_bias): a stable sort
+                    roster = np.lexsort((np.arange(16), -counts[t]))[:m]
+                    assert all(int(e) in roster for e in idx[t])
+                    seen_after_pin[t].update(int(e) for e in idx[t])
+            oracle.roster_update(counts, idx, lib=lib)
+        used[delta] = np.mean([(c > 0).sum() for c in counts])
+        if delta > 0:
+            assert max(len(v) for v in seen_after_pin) <= m
+    # the unbiased router spreads each sequence over many more experts than the budget
+    assert used[0.0] > 2 * m and used[0.05] < used[0.0], used
+
+
 PINS = [pin_keep_count, pin_gate_matches_library, pin_select_bruteforce, pin_threshold_strict,
         pin_routing, pin_dense_at_zero_sparsity, pin_masked_layer, pin_invariants,
-        pin_calibration]
+        pin_calibration, pin_roster_bias, pin_route_biased, pin_roster_sequences]
 
 
 def run_all(lib):

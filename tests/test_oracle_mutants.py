@@ -41,6 +41,14 @@ MUTANTS = [
     ("calibration_ceil", "(long long)floor(s * (double)N)", "(long long)ceil(s * (double)N)", 0),
     ("shared_uses_routed_sparsity", "      sel = shared;", "      sel = routed;", 0),
     ("h_from_g_not_silu", "keep, a.data(), &y", "keep, g.data(), &y", 0),
+    ("roster_bias_on_weights", "route_weights(*L, lg.data(), idx + (size_t)t * k",
+     "route_weights(*L, sel.data(), idx + (size_t)t * k", 0),
+    ("roster_tie_reversed", "return p < q;", "return p > q;", 2),
+    ("roster_no_exploration", "else if (distinct < m)", "else if (distinct < 0)", 0),
+    ("roster_barrier_sign", "b[e] = member[e] ? delta : -delta;",
+     "b[e] = member[e] ? -delta : delta;", 0),
+    ("roster_pin_ignored", "if (pinned[t]) b[e]", "if (pinned[t] && 0) b[e]", 0),
+    ("roster_update_ignored", "counts[(size_t)t * E + e] += 1;", "counts[(size_t)t * E + e] += 0;", 0),
 ]
 
 
