@@ -1,14 +1,18 @@
 """Benchmark of the sparse-expert MoE FFN decode layer on B200.
 
 One step = one layer call (router, gate, selection, sparse up/down, output cast) on one batch
-of synthetic decode tokens.  Default workload: the OLMoE-shaped bf16 layer (H2048, 64 experts,
-top-8, I1024) at 16 tokens and 90 % intra-expert sparsity; ``--sweep`` adds the batch x
-sparsity grid (1..256 tokens, s = 0 / 0.5 / 0.9).  L2 is flushed (a 2x-L2 buffer is written,
-then another is read) before every timed step and the token batch rotates through a pool of 32.
-The line also reports the same steps replayed from CUDA graphs (``graph``) and through the
-host-buffer call with its copies (``e2e``).
+of synthetic decode tokens.  Default workload: the Llama-4-Maverick-shaped bf16 layer (H5120,
+128 routed experts top-1 with a sigmoid gate, one shared expert, I = Ish = 8192; about 32 GB of
+expert weights resident) at 16 tokens and 90 % intra-expert sparsity for routed and shared
+experts.  ``--sweep`` (on by default on one GPU) adds the metric's grid on every bf16 shape:
+Llama-4 at 1..256 tokens, OLMoE at 1..256, DeepSeek-V2-Lite at 1..64 with shared-expert sparsity
+0 and 0.5, GPT-OSS-120B at 1..64 in top-K mode and in threshold mode; sparsity 0 / 0.5 / 0.9.
+L2 is flushed (a 2x-L2 buffer is written, then another is read) before every timed step and the
+token batch rotates through a pool of 32.  The line also reports the same steps replayed from
+CUDA graphs (``graph``) and through the host-buffer call with its copies (``e2e``).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cuda|reference]
+                  [--workload llama4|olmoe|dsv2l|gptoss] [--batch B] [--sparsity s]
 
 Multi-GPU: one process per GPU (torchrun); each rank runs the layer on its own token batches
 (independent decode streams, no data-path collective), so per-GPU work is fixed: weak scaling.
@@ -36,6 +40,24 @@ HBM_SPEC_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 DEFAULT_DENSE_MIN = -1  # the library's default: automatic path choice per call
 
+# command-line names of the workload shapes
+WORKLOADS = {"llama4": "llama4-maverick", "olmoe": "olmoe", "dsv2l": "dsv2-lite",
+             "gptoss": "gpt-oss-120b", "tiny": "tiny-fp32"}
+
+# The metric's grid: (shape, batches, [(selection, routed s, shared s)]).  Threshold rows carry
+# the target sparsity the threshold is calibrated for.
+SWEEP = [
+    ("llama4-maverick", [1, 2, 4, 8, 16, 32, 64, 128, 256],
+     [("topk", s, s) for s in (0.0, 0.5, 0.9)]),
+    ("olmoe", [1, 4, 16, 64, 256], [("topk", s, None) for s in (0.0, 0.5, 0.9)]),
+    ("dsv2-lite", [1, 2, 4, 8, 16, 32, 64],
+     [("topk", s, sh) for sh in (0.0, 0.5) for s in (0.0, 0.5, 0.9)]),
+    ("gpt-oss-120b", [1, 8, 32, 64],
+     [("topk", s, None) for s in (0.0, 0.5, 0.9)] +
+     [("threshold", s, None) for s in (0.5, 0.9)]),
+]
+CALIB_TOKENS = 1024  # threshold calibration tokens (seeded apart from the token stream)
+
 
 def parse():
     ap = argparse.ArgumentParser()
@@ -43,7 +65,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
-    ap.add_argument("--workload", default="olmoe")
+    ap.add_argument("--workload", default="llama4")
     ap.add_argument("--batch", type=int, default=16)
     ap.add_argument("--sparsity", type=float, default=0.9)
     ap.add_argument("--sweep", dest="sweep", action="store_true", default=None)
@@ -167,31 +189,36 @@ def workload_config(shape, B, world, s):
     return {"workload": f"{shape.name}-shaped MoE layer", "hidden": shape.hidden,
             "experts": shape.n_routed, "top_k": shape.top_k, "inter": shape.inter,
             "shared": shape.n_shared, "batch_per_gpu": B, "global_batch": B * world,
-            "sparsity": s, "selection": "top-K per (token, expert)"}
+            "sparsity": s, "selection": "top-K per (token, expert)"
+            + (", the same sparsity for the shared experts" if shape.n_shared else "")}
+
+
+def shape_of(name):
+    import synth
+    return synth.SHAPES[WORKLOADS.get(name, name)]
 
 
 def algorithmic_bytes(shape, dbg, B):
     """Bytes the method must read per stage for one call (each touched expert's gate block
     once, each kept row of the per-expert union once), from the call's kept lists."""
+    import numpy as np
     elt, H = shape.elt, shape.hidden
     k, S = shape.top_k, shape.n_shared
-    union = {}
-    for t in range(B):
-        for j in range(k):
-            e = int(dbg["idx"][t][j])
-            kept = dbg["lists"][t][j][: dbg["cnt"][t][j]]
-            union.setdefault(("r", e), set()).update(kept.tolist())
-        for s in range(S):
-            union.setdefault(("s", s), set()).update(
-                dbg["lists"][t][k + s][: dbg["cnt"][t][k + s]].tolist())
-    gate = sum((shape.inter if kind == "r" else shape.inter_shared) * H * elt
-               for (kind, _) in union)
-    updown = sum(len(u) * 2 * H * elt for u in union.values())
-    pairs = B * (k + S)
     imax = max(shape.inter, shape.inter_shared if S else 0)
+    idx = np.asarray(dbg["idx"][:B])
+    routed = sorted(set(int(e) for e in idx.ravel()))
+    row_of = {e: i for i, e in enumerate(routed)}
+    union = np.zeros((len(routed) + S, imax + 1), bool)  # column imax absorbs the -1 padding
+    for t in range(B):
+        for j in range(k + S):
+            u = row_of[int(idx[t][j])] if j < k else len(routed) + j - k
+            union[u, dbg["lists"][t][j][: int(dbg["cnt"][t][j])]] = True
+    rows = int(union[:, :imax].sum())
+    gate = (len(routed) * shape.inter + S * shape.inter_shared) * H * elt
+    pairs = B * (k + S)
     return {"router": shape.n_routed * H * elt + B * H * elt, "gate": gate,
-            "select": pairs * imax * 4, "updown": updown, "finalize": B * H * (8 + elt),
-            "rows": sum(len(u) for u in union.values())}
+            "select": pairs * imax * 4, "updown": rows * 2 * H * elt,
+            "finalize": B * H * (8 + elt), "rows": rows}
 
 
 def traffic_of(key):
@@ -233,6 +260,111 @@ def token_stream(rank, i):
     return rank * 1000 + i
 
 
+def make_flush(dev):
+    """Writes a 2x-L2 buffer, then reads another one, so that the next timed step starts with
+    an L2 that holds none of the layer's data and no dirty lines to write back."""
+    import torch
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_w = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=dev)
+    flush_r = torch.ones_like(flush_w)
+
+    def flush():
+        flush_w.zero_()
+        flush_r.sum()
+    return flush
+
+
+def timed_calls(dl, batches, rule_r, rule_s, steps, warmup, flush, out):
+    """Event-timed layer calls (ms each), the L2 flushed before each, batches rotating."""
+    import torch
+    for i in range(warmup):
+        dl.forward(batches[i % len(batches)], rule_r, rule_s, out=out)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for i in range(steps):
+        flush()
+        evs[i][0].record()
+        dl.forward(batches[i % len(batches)], rule_r, rule_s, out=out)
+        evs[i][1].record()
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def calibrate_threshold(dl, s, chunk):
+    """Threshold t for target sparsity s from the layer's own fp32 activations of the routed
+    pairs of CALIB_TOKENS seeded calibration tokens: the scores |SiLU(g)| sorted ascending as
+    S[0..N), t = S[m - 1] with m = floor(s N), so that the top N - m scores exceed it (the same
+    order statistic as the tests' fp64 calibration; here the scores are the device's)."""
+    import torch
+
+    import synth
+    shape = dl.shape
+    xs = dl.tokens(CALIB_TOKENS, synth.calib_seed(shape))
+    scores = []
+    for c0 in range(0, CALIB_TOKENS, chunk):
+        x = xs[c0:c0 + chunk].contiguous()
+        n = x.shape[0]
+        dl.forward(x, ("topk", 0.0), ("topk", 0.0))
+        d = dl.debug_device(n)
+        scores.append(d["act"][:, :shape.top_k, :shape.inter].abs().reshape(-1))
+    allv = torch.cat(scores)
+    m = int(s * allv.numel())
+    if m == 0:
+        return float("-inf")
+    return float(torch.kthvalue(allv.cpu(), m).values)
+
+
+def sweep_rows(dl, batches, rules, peak, flush, pool_n, token_stream_of, steps=20):
+    """The metric's grid on one shape: per (batch, rule) the median layer time, tokens/s and
+    the active-weight bytes over time against the HBM peak; the s = 0.9 / s = 0 speed-up per
+    batch and shared-expert sparsity."""
+    import torch
+
+    import synth
+    shape = dl.shape
+    rows = []
+    thresholds = {}
+    for kind, s, s_sh in rules:
+        if kind == "threshold" and s not in thresholds:
+            thresholds[s] = calibrate_threshold(dl, s, max(batches))
+    for B in batches:
+        bx = [dl.tokens(B, synth.token_seed(shape, token_stream_of(i))) for i in range(pool_n)]
+        out = torch.empty_like(bx[0])
+        times = {}
+        for kind, s, s_sh in rules:
+            if kind == "threshold":
+                r_r = ("threshold", thresholds[s])
+                r_s = r_r if shape.n_shared else None
+            else:
+                r_r = ("topk", s)
+                r_s = ("topk", s_sh) if shape.n_shared else None
+            ms = statistics.median(timed_calls(dl, bx, r_r, r_s, steps, 3, flush, out))
+            nbytes, nrep = 0.0, 2
+            for i in range(nrep):
+                dl.forward(bx[i], r_r, r_s, out=out)
+                ab = algorithmic_bytes(shape, dl.debug(B), B)
+                nbytes += (ab["router"] + ab["gate"] + ab["updown"]) / nrep
+            gbs = nbytes / (ms / 1e3) / 1e9
+            row = {"workload": shape.name, "batch": B, "selection": kind, "sparsity": s}
+            if shape.n_shared:
+                row["shared_sparsity"] = s_sh
+            if kind == "threshold":
+                row["threshold"] = thresholds[s]
+            row.update({"us": round(ms * 1e3, 1), "tokens_per_s": round(B / (ms / 1e3), 1),
+                        "tokens_per_expert": round(B * shape.top_k / shape.n_routed, 3),
+                        "launches": dl.last_launches(),
+                        "active_bytes": int(nbytes), "gbs": round(gbs, 1),
+                        "frac": round(gbs / peak, 4), "frac_spec": round(gbs / HBM_SPEC_GBS, 4)})
+            rows.append(row)
+            times[(kind, s, s_sh)] = (ms, row)
+        for (kind, s, s_sh), (ms, row) in times.items():
+            if kind == "topk" and s == 0.9 and ("topk", 0.0, s_sh) in times:
+                row["speedup_s0.9_vs_s0"] = round(times[("topk", 0.0, s_sh)][0] / ms, 3)
+        del bx, out
+    return rows
+
+
 def run_cuda(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -244,12 +376,13 @@ def run_cuda(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    shape = synth.SHAPES[args.workload]
+    shape = shape_of(args.workload)
     B, s = args.batch, args.sparsity
     sweep_on = args.sweep if args.sweep is not None else (world == 1)
-    sweep_B = [1, 4, 16, 64, 256] if sweep_on else []
-    max_tokens = max([B] + sweep_B)
+    plan = {name: (bs, rules) for name, bs, rules in SWEEP} if sweep_on else {}
+    max_tokens = max([B] + (plan[shape.name][0] if shape.name in plan else []))
     rule = ("topk", s)
+    rule_s = rule if shape.n_shared else None
     dl = DeviceLayer(shape, max_tokens=max_tokens, device=dev)
     pool_n = 32
 
@@ -259,39 +392,11 @@ def run_cuda(args, rank, world, local_rank):
 
     xs = pool(B)
     out = torch.empty_like(xs[0])
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush_w = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=dev)
-    flush_r = torch.ones_like(flush_w)
+    flush = make_flush(dev)
 
-    class _Flush:
-        """Writes a 2x-L2 buffer, then reads another one, so that the timed step starts with
-        an L2 that holds none of the layer's data and no dirty lines to write back."""
-
-        @staticmethod
-        def zero_():
-            flush_w.zero_()
-            flush_r.sum()
-
-    flush = _Flush()
-
-    def timed(batches, rule_, steps, warmup):
-        for i in range(warmup):
-            dl.forward(batches[i % len(batches)], rule_, rule_, out=out_b[id(batches)])
-        torch.cuda.synchronize()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(steps)]
-        for i in range(steps):
-            flush.zero_()
-            evs[i][0].record()
-            dl.forward(batches[i % len(batches)], rule_, rule_, out=out_b[id(batches)])
-            evs[i][1].record()
-        torch.cuda.synchronize()
-        return [a.elapsed_time(b) for a, b in evs]
-
-    out_b = {id(xs): out}
     # ---- the timed run (warm-up, barrier, K steps, barrier)
     for i in range(args.warmup):
-        dl.forward(xs[i % pool_n], rule, rule, out=out)
+        dl.forward(xs[i % pool_n], rule, rule_s, out=out)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -304,15 +409,16 @@ def run_cuda(args, rank, world, local_rank):
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     for i in range(args.steps):
-        flush.zero_()
+        flush()
         evs[i][0].record()
-        dl.forward(xs[i % pool_n], rule, rule, out=out)
+        dl.forward(xs[i % pool_n], rule, rule_s, out=out)
         evs[i][1].record()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clock_info = clocks.stop()
+    launches = dl.last_launches()
     step_ms = [a.elapsed_time(b) for a, b in evs]
     total_ms = job_time_ms(sum(step_ms), world, dev)
     value = job_throughput(world, B, args.steps, total_ms)
@@ -326,16 +432,16 @@ def run_cuda(args, rank, world, local_rank):
     stage_ms = {n: [] for n in STAGES}
     nprof = min(args.steps, 20)
     for i in range(nprof):
-        flush.zero_()
-        dl.forward(xs[i % pool_n], rule, rule, out=out)
+        flush()
+        dl.forward(xs[i % pool_n], rule, rule_s, out=out)
         torch.cuda.synchronize()
         for j, n in enumerate(STAGES):
             stage_ms[n].append(stage_evs[j].elapsed_time(stage_evs[j + 1]))
     moe_profile_stages(dl.h, None)
     abytes = {n: 0.0 for n in STAGES}
-    nb = min(pool_n, nprof)
+    nb = min(pool_n, nprof, 8)
     for i in range(nb):
-        dl.forward(xs[i], rule, rule, out=out)
+        dl.forward(xs[i], rule, rule_s, out=out)
         ab = algorithmic_bytes(shape, dl.debug(B), B)
         for n in STAGES:
             abytes[n] += ab[n] / nb
@@ -344,7 +450,7 @@ def run_cuda(args, rank, world, local_rank):
     peak, peak_kind = peaks()
     achieved = abytes[dom] / (stage_avg[dom] / 1e3) / 1e9
     layer_bytes = sum(abytes[n] for n in ("router", "gate", "updown"))
-    traffic = traffic_of(f"{args.workload}:B{B}:s{s}:{dom}")
+    traffic = traffic_of(f"{shape.name}:B{B}:s{s}:{dom}")
     layer_gbs = layer_bytes / (total_ms / args.steps / 1e3) / 1e9
     roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
                 "peak_source": f"hbm copy, {peak_kind}", "unit": "GB/s",
@@ -368,7 +474,7 @@ def run_cuda(args, rank, world, local_rank):
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
     for i in range(args.steps):
-        flush.zero_()
+        flush()
         e2e_ev[i][0].record()
         moe_forward_host(dl.h, xh[i % 8], B, dl.router, dl.routed, dl.shared, sr, ss, oh)
         e2e_ev[i][1].record()
@@ -380,18 +486,18 @@ def run_cuda(args, rank, world, local_rank):
            "api": "moe_forward_host"}
 
     # ---- the same steps replayed from CUDA graphs: one captured layer call per pooled batch
-    # (the five launches and their programmatic edges are recorded once, replayed per step)
+    # (the launches and their programmatic edges are recorded once, replayed per step)
     side = torch.cuda.Stream(device=dev)
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):
-        dl.forward(xs[0], rule, rule, out=out)
+        dl.forward(xs[0], rule, rule_s, out=out)
     torch.cuda.current_stream().wait_stream(side)
     torch.cuda.synchronize()
     graphs = []
     for i in range(pool_n):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            dl.forward(xs[i], rule, rule, out=out)
+            dl.forward(xs[i], rule, rule_s, out=out)
         graphs.append(g)
     for i in range(args.warmup):
         graphs[i % pool_n].replay()
@@ -399,7 +505,7 @@ def run_cuda(args, rank, world, local_rank):
     g_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             for _ in range(args.steps)]
     for i in range(args.steps):
-        flush.zero_()
+        flush()
         g_ev[i][0].record()
         graphs[i % pool_n].replay()
         g_ev[i][1].record()
@@ -409,31 +515,22 @@ def run_cuda(args, rank, world, local_rank):
              "ms_per_step": round(g_ms / args.steps, 5), "graphs": pool_n}
     del graphs
 
-    # ---- sweep (rank 0, single GPU)
+    # ---- sweep (rank 0, single GPU): the metric's grid on every bf16 shape
     sweep = []
     if sweep_on and rank == 0:
-        for sb in sweep_B:
-            bx = pool(sb)
-            out_b[id(bx)] = torch.empty_like(bx[0])
-            row = {}
-            for ss_ in (0.0, 0.5, 0.9):
-                r_ = ("topk", ss_)
-                ms = timed(bx, r_, 20, 3)
-                med = statistics.median(ms)
-                nbytes = 0.0
-                for i in range(4):
-                    dl.forward(bx[i], r_, r_, out=out_b[id(bx)])
-                    ab = algorithmic_bytes(shape, dl.debug(sb), sb)
-                    nbytes += (ab["router"] + ab["gate"] + ab["updown"]) / 4
-                gbs = nbytes / (med / 1e3) / 1e9
-                row[ss_] = med
-                sweep.append({"batch": sb, "sparsity": ss_, "us": round(med * 1e3, 1),
-                              "tokens_per_s": round(sb / (med / 1e3), 1),
-                              "active_bytes": int(nbytes), "gbs": round(gbs, 1),
-                              "frac": round(gbs / peak, 4),
-                              "frac_spec": round(gbs / HBM_SPEC_GBS, 4)})
-            sweep[-1]["speedup_s0.9_vs_s0"] = round(row[0.0] / row[0.9], 3)
-            del out_b[id(bx)]
+        for name, bs, rules in SWEEP:
+            if name == shape.name:
+                sdl = dl
+            else:
+                sdl = DeviceLayer(synth.SHAPES[name], max_tokens=max(bs), device=dev)
+            try:
+                sweep += sweep_rows(sdl, bs, rules, peak, flush, pool_n,
+                                    lambda i: token_stream(rank, i))
+            finally:
+                if sdl is not dl:
+                    sdl.close()
+                    del sdl
+                    torch.cuda.empty_cache()
 
     # ---- CPU baseline: the oracle, as it stands, on a bounded sample (rank 0, N = 1)
     cpu = None
@@ -450,90 +547,127 @@ def run_cuda(args, rank, world, local_rank):
                               "2x-L2 buffer read (clean lines, none of the layer's)",
                            token_pool=pool_n, parallelism=f"replicas x{world}"),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "graph": graph,
-            "gpu_launches": 5 * args.steps, "clocks": clock_info}
+            "gpu_launches": launches * args.steps, "clocks": clock_info}
     if sweep:
         line["sweep"] = sweep
     return line
 
 
 # ---------------------------------------------------------------------------------------------
+class OracleSample:
+    """Token batches of the benchmark's workload for the fp64 oracle, with their weights.
+
+    Batches hold min(B, 8) tokens of the bench's token streams when the shape's routed weights
+    exceed 4 GB (the Llama-4 shape: the oracle then holds a fixed set of 16 routed experts and
+    draws only tokens routed among them, so that host memory stays bounded; the oracle's cost
+    per token does not depend on which expert it routes to), else B tokens with every expert's
+    weights drawn when first needed."""
+
+    def __init__(self, shape, B, stream0=0):
+        import oracle
+        import synth
+        self.shape, self.synth, self.oracle = shape, synth, oracle
+        routed_bytes = shape.n_routed * 3 * shape.inter * shape.hidden * shape.elt
+        self.limited = routed_bytes > (4 << 30)
+        self.nb = min(B, 8) if self.limited else B
+        self.router = synth.host_tensor(shape, "router")
+        self.rl = oracle.Layer(shape, self.router, {}, [])
+        self.shared = [(synth.host_tensor(shape, "sh_gate", j), synth.host_tensor(shape, "sh_up", j),
+                        synth.host_tensor(shape, "sh_down", j)) for j in range(shape.n_shared)]
+        self.cache = {}
+        self.stream = stream0
+        self.pending = []
+
+    def _expert(self, e):
+        s = self.synth
+        if e not in self.cache:
+            self.cache[e] = (s.host_tensor(self.shape, "gate", e), s.host_tensor(self.shape, "up", e),
+                             s.host_tensor(self.shape, "down", e))
+        return self.cache[e]
+
+    def next(self):
+        """(layer, x) of the next batch; drawing weights is not part of the oracle's time."""
+        import numpy as np
+        s = self.synth
+        if not self.limited:
+            x = s.host_tokens(self.shape, self.nb, s.token_seed(self.shape, self.stream))
+            self.stream += 1
+            _, idx, _ = self.rl.route(x)
+            need = sorted(set(int(e) for e in idx.ravel()))
+            return self.oracle.Layer(self.shape, self.router, {e: self._expert(e) for e in need},
+                                     self.shared), x
+        while len(self.pending) < self.nb:
+            x = s.host_tokens(self.shape, 64, s.token_seed(self.shape, self.stream))
+            self.stream += 1
+            _, idx, _ = self.rl.route(x)
+            for t in range(x.shape[0]):
+                es = [int(e) for e in idx[t]]
+                if len(self.cache) < 16:
+                    for e in es:
+                        self._expert(e)
+                if all(e in self.cache for e in es):
+                    self.pending.append(x[t])
+        x = np.stack(self.pending[:self.nb])
+        self.pending = self.pending[self.nb:]
+        return self.oracle.Layer(self.shape, self.router, dict(self.cache), self.shared), x
+
+    def describe(self):
+        if self.limited:
+            return (f"batches of {self.nb} tokens of the token streams routed among a fixed set "
+                    f"of 16 routed experts (host memory bound)")
+        return f"batches of {self.nb} tokens of the token streams"
+
+
 def cpu_baseline(shape, B, rule, seconds):
-    """Times the fp64 oracle (all host cores) on whole token batches of the benchmark's stream,
+    """Times the fp64 oracle (all host cores) on batches of the benchmark's token streams,
     batch after batch, until about `seconds` of oracle time has been spent."""
-    import oracle
-    import synth
-    router = synth.host_tensor(shape, "router")
-    rl = oracle.Layer(shape, router, {}, [])
-    shared = [(synth.host_tensor(shape, "sh_gate", j), synth.host_tensor(shape, "sh_up", j),
-               synth.host_tensor(shape, "sh_down", j)) for j in range(shape.n_shared)]
-    cache = {}
+    rule_s = rule if shape.n_shared else None
+    smp = OracleSample(shape, B)
     done_tok, spent, nb = 0, 0.0, 0
     while spent < seconds and nb < 4096:
-        x = synth.host_tokens(shape, B, synth.token_seed(shape, nb))
-        _, idx, _ = rl.route(x)
-        need = sorted(set(int(e) for e in idx.ravel()))
-        for e in need:
-            if e not in cache:
-                cache[e] = (synth.host_tensor(shape, "gate", e), synth.host_tensor(shape, "up", e),
-                            synth.host_tensor(shape, "down", e))
-        lay = oracle.Layer(shape, router, {e: cache[e] for e in need}, shared)
+        lay, x = smp.next()
         t0 = time.perf_counter()
-        lay.forward(x, rule, rule)
+        lay.forward(x, rule, rule_s)
         spent += time.perf_counter() - t0
-        done_tok += B
+        done_tok += x.shape[0]
         nb += 1
-    return {"value": round(done_tok / spent, 3), "unit": UNIT, "cores": oracle.threads(),
+    return {"value": round(done_tok / spent, 3), "unit": UNIT, "cores": smp.oracle.threads(),
             "kind": "oracle",
-            "sample": f"{nb} batches of {B} tokens (token streams 1..{nb}), whole layer in fp64, "
-                      f"{spent:.1f} s of oracle time"}
+            "sample": f"{nb} {smp.describe()}, whole layer in fp64, {spent:.1f} s of oracle time"}
 
 
 def run_reference(args):
     """The benchmark's reference arm: the fp64 CPU oracle, timed on the host cores."""
-    import synth
-    shape = synth.SHAPES[args.workload]
+    shape = shape_of(args.workload)
     B, rule = args.batch, ("topk", args.sparsity)
+    rule_s = rule if shape.n_shared else None
+    smp = OracleSample(shape, B)
+    batches = [smp.next() for _ in range(4)]
+    # tokens per step: sized so that the whole run stays within a few minutes
     per_step = max(1.0, args.cpu_seconds / max(1, args.steps + args.warmup) * 4)
-    import oracle
-    x_all = [synth.host_tokens(shape, B, synth.token_seed(shape, i)) for i in range(4)]
-    router = synth.host_tensor(shape, "router")
-    rl = oracle.Layer(shape, router, {}, [])
-    shared = [(synth.host_tensor(shape, "sh_gate", j), synth.host_tensor(shape, "sh_up", j),
-               synth.host_tensor(shape, "sh_down", j)) for j in range(shape.n_shared)]
-    cache = {}
-
-    def layer_for(x):
-        _, idx, _ = rl.route(x)
-        need = sorted(set(int(e) for e in idx.ravel()))
-        for e in need:
-            if e not in cache:
-                cache[e] = (synth.host_tensor(shape, "gate", e), synth.host_tensor(shape, "up", e),
-                            synth.host_tensor(shape, "down", e))
-        return oracle.Layer(shape, router, {e: cache[e] for e in need}, shared)
-
-    # tokens per step: sized so the whole run stays within a few minutes
-    probe = layer_for(x_all[0][:1])
+    lay0, x0 = batches[0]
     t0 = time.perf_counter()
-    probe.forward(x_all[0][:1], rule, rule)
+    lay0.forward(x0[:1], rule, rule_s)
     one = time.perf_counter() - t0
-    ntok = int(max(1, min(B, per_step / max(one, 1e-6))))
-    layers = [layer_for(x[:ntok]) for x in x_all]
+    ntok = int(max(1, min(smp.nb, per_step / max(one, 1e-6))))
     for i in range(args.warmup):
-        layers[i % 4].forward(x_all[i % 4][:ntok], rule, rule)
+        lay, x = batches[i % 4]
+        lay.forward(x[:ntok], rule, rule_s)
     t0 = time.perf_counter()
     for i in range(args.steps):
-        layers[i % 4].forward(x_all[i % 4][:ntok], rule, rule)
+        lay, x = batches[i % 4]
+        lay.forward(x[:ntok], rule, rule_s)
     dt = time.perf_counter() - t0
     value = ntok * args.steps / dt
-    sample = f"{ntok} of {B} tokens per step, whole layer in fp64"
+    sample = f"{ntok} tokens per step from {smp.describe()}, whole layer in fp64"
     return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": dict(workload_config(shape, B, args.gpus, args.sparsity),
-                           token_pool=len(x_all), parallelism="host cores"),
-            "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": oracle.threads(),
-                             "kind": "oracle", "sample": sample},
+                           token_pool=4, parallelism="host cores"),
+            "cpu_baseline": {"value": round(value, 3), "unit": UNIT,
+                             "cores": smp.oracle.threads(), "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
@@ -547,36 +681,24 @@ def run_crossover(args):
     import synth
     from sparse_expert_ffn_logits_b200 import moe_set_dense_min_tokens
     from sparse_expert_ffn_logits_b200.workload import DeviceLayer
-    shape = synth.SHAPES[args.workload]
-    batches = [b for b in (8, 16, 32, 64, 128, 256)]
+    shape = shape_of(args.workload)
+    batches = [1, 2, 4, 8, 16, 32, 64, 128, 256]
     dl = DeviceLayer(shape, max_tokens=max(batches))
-    default_min = DEFAULT_DENSE_MIN
-    l2 = torch.cuda.get_device_properties(0).L2_cache_size
-    flush_w = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device="cuda")
-    flush_r = torch.ones_like(flush_w)
+    flush = make_flush(torch.device("cuda", 0))
     rows = []
     for B in batches:
         xs = [dl.tokens(B, synth.token_seed(shape, 500 + i)) for i in range(8)]
         out = torch.empty_like(xs[0])
         for s in (0.0, 0.5, 0.9):
             rule = ("topk", s)
+            rule_s = rule if shape.n_shared else None
             t = {}
-            for name, dmin in (("sparse", 0), ("dense", 1), ("auto", default_min)):
+            for name, dmin in (("sparse", 0), ("dense", 1), ("auto", DEFAULT_DENSE_MIN)):
                 moe_set_dense_min_tokens(dl.h, dmin)
-                for i in range(3):
-                    dl.forward(xs[i], rule, rule, out=out)
-                ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                      for _ in range(args.steps)]
-                for i in range(args.steps):
-                    flush_w.zero_()
-                    flush_r.sum()
-                    ev[i][0].record()
-                    dl.forward(xs[i % len(xs)], rule, rule, out=out)
-                    ev[i][1].record()
-                torch.cuda.synchronize()
-                t[name] = statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3
+                t[name] = statistics.median(
+                    timed_calls(dl, xs, rule, rule_s, args.steps, 3, flush, out)) * 1e3
             row = {"workload": shape.name, "batch": B, "sparsity": s,
-                   "tokens_per_expert": round(B * shape.top_k / shape.n_routed, 2),
+                   "tokens_per_expert": round(B * shape.top_k / shape.n_routed, 3),
                    "sparse_us": round(t["sparse"], 1), "dense_us": round(t["dense"], 1),
                    "auto_us": round(t["auto"], 1),
                    "faster": "dense" if t["dense"] < t["sparse"] else "sparse"}

@@ -130,6 +130,36 @@ moe_status moe_forward(moe_handle* h, const void* x, int n_tokens, const void* r
                        const moe_sparsity* sp_routed, const moe_sparsity* sp_shared, void* out,
                        void* stream);
 
+/* Roster routing state of the batch's sequences ("Predatory MoE", technical summary,
+ * Methodology 2, the roster rule), one row per token: token t of a call is the decode token of
+ * the sequence whose state is row t.
+ *   counts  [n_tokens][E] int32, device, read and updated: how often each expert of this layer
+ *           was selected for the sequence so far (the call adds its own choice)
+ *   pinned  [n_tokens] int32, device, read: nonzero = the sequence's roster is pinned
+ *   m       roster budget, top_k <= m <= E
+ *   delta   barrier bonus, finite and >= 0
+ * The roster of a sequence is its m most-selected experts (equal counts: lower index).  While
+ * fewer than m distinct experts have been selected the router is unchanged (exploration); then
+ * the choice is the top-k of logit + delta for members and logit - delta for the others; a
+ * pinned sequence chooses among its roster only.  The bias acts on the choice: the routing
+ * weights are those of the unbiased logits of the chosen experts. */
+typedef struct {
+  int* counts;
+  const int* pinned;
+  int m;
+  float delta;
+} moe_roster;
+
+/* moe_forward with roster routing (one more kernel before the router computes each sequence's
+ * bias; the router adds the choice to the counts).  INVALID_ARG for a NULL roster or buffer, a
+ * buffer that is not 4-byte aligned, m outside [top_k, E] or a negative or non-finite delta;
+ * otherwise as moe_forward.  The calls of one decode step must not overlap on the GPU with
+ * another call that updates the same counts. */
+moe_status moe_forward_roster(moe_handle* h, const void* x, int n_tokens, const void* router,
+                              const moe_roster* roster, const moe_expert_weights* routed,
+                              const moe_expert_weights* shared, const moe_sparsity* sp_routed,
+                              const moe_sparsity* sp_shared, void* out, void* stream);
+
 /* moe_forward with x and out in HOST memory: copies x to the handle's device staging buffer,
  * runs the layer and copies the result back, all asynchronously on `stream` (page-locked host
  * buffers make the copies asynchronous; the caller synchronises the stream before reading
@@ -195,6 +225,11 @@ moe_status moe_debug_force_timeout(moe_handle* h, void* stream);
  * INVALID_ARG for a NULL handle or a value below -1.  Takes effect from the next moe_forward. */
 #define MOE_DENSE_AUTO (-1)
 moe_status moe_set_dense_min_tokens(moe_handle* h, int min_tokens);
+
+/* How many kernels the last successful moe_forward on this handle launched (5 on the sparse
+ * path: router, gate, select, up/down, output cast; 9 when the tensor-core path ran as well;
+ * one more with roster routing; 0 before the first call).  Host-side only: reads no device memory.  INVALID_ARG for NULL. */
+moe_status moe_last_launches(moe_handle* h, int* n);
 
 /* Frees the workspace and the handle (synchronises the device first).  NULL is a no-op. */
 moe_status moe_destroy(moe_handle* h);

@@ -42,6 +42,11 @@ class MoESparsity(ctypes.Structure):
                 ("threshold", ctypes.c_float)]
 
 
+class MoERoster(ctypes.Structure):
+    _fields_ = [("counts", ctypes.c_void_p), ("pinned", ctypes.c_void_p), ("m", ctypes.c_int),
+                ("delta", ctypes.c_float)]
+
+
 class MoEExpertWeights(ctypes.Structure):
     _fields_ = [("gate", ctypes.c_void_p), ("updown", ctypes.c_void_p)]
 
@@ -50,8 +55,10 @@ _LIB = None
 
 # C entry points declared in include/moe.h
 EXPORTS = ("moe_create", "moe_packed_bytes", "moe_pack_experts", "moe_forward",
+           "moe_forward_roster",
            "moe_forward_host", "moe_debug_lists", "moe_profile_stages", "moe_read_trace",
-           "moe_get_error", "moe_debug_force_timeout", "moe_set_dense_min_tokens", "moe_destroy",
+           "moe_get_error", "moe_debug_force_timeout", "moe_set_dense_min_tokens",
+           "moe_last_launches", "moe_destroy",
            "moe_route_noalloc",
            "moe_status_string")
 MOE_STAGE_EVENTS = 6
@@ -75,12 +82,18 @@ def _lib():
                ctypes.POINTER(MoESparsity), ctypes.POINTER(MoESparsity), P, P]
         lib.moe_forward.argtypes = fwd
         lib.moe_forward_host.argtypes = fwd
+        lib.moe_forward_roster.argtypes = [P, P, I, P, ctypes.POINTER(MoERoster),
+                                           ctypes.POINTER(MoEExpertWeights),
+                                           ctypes.POINTER(MoEExpertWeights),
+                                           ctypes.POINTER(MoESparsity), ctypes.POINTER(MoESparsity),
+                                           P, P]
         lib.moe_debug_lists.argtypes = [P, I, P, P, P, P, P, P, P]
         lib.moe_profile_stages.argtypes = [P, ctypes.POINTER(P), I]
         lib.moe_read_trace.argtypes = [P, P, ctypes.c_size_t]
         lib.moe_get_error.argtypes = [P, ctypes.POINTER(I)]
         lib.moe_destroy.argtypes = [P]
         lib.moe_set_dense_min_tokens.argtypes = [P, I]
+        lib.moe_last_launches.argtypes = [P, ctypes.POINTER(I)]
         lib.moe_debug_force_timeout.argtypes = [P, P]
         lib.moe_route_noalloc.argtypes = [ctypes.POINTER(MoEConfig), P, I, P, P, P, P]
         lib.moe_status_string.argtypes = [I]
@@ -165,6 +178,21 @@ def moe_forward(h, x, n_tokens, router, routed, shared, sp_routed, sp_shared, ou
                               _ptr(out), _stream(stream)), "moe_forward")
 
 
+def roster(counts, pinned, m, delta):
+    """MoERoster over device int32 tensors counts [B][E] and pinned [B]."""
+    return MoERoster(_ptr(counts), _ptr(pinned), int(m), float(delta))
+
+
+def moe_forward_roster(h, x, n_tokens, router, roster_state, routed, shared, sp_routed,
+                       sp_shared, out, stream=None):
+    _check(_lib().moe_forward_roster(ctypes.c_void_p(h), _ptr(x), int(n_tokens), _ptr(router),
+                                     ctypes.byref(roster_state), ctypes.byref(routed),
+                                     ctypes.byref(shared) if shared else None,
+                                     ctypes.byref(sp_routed),
+                                     ctypes.byref(sp_shared) if sp_shared else None, _ptr(out),
+                                     _stream(stream)), "moe_forward_roster")
+
+
 def moe_forward_host(h, x_host, n_tokens, router, routed, shared, sp_routed, sp_shared, out_host,
                      stream=None):
     _check(_lib().moe_forward_host(ctypes.c_void_p(h), _ptr(x_host), int(n_tokens), _ptr(router),
@@ -224,6 +252,14 @@ def moe_set_dense_min_tokens(h, min_tokens):
     token threshold (see include/moe.h)."""
     _check(_lib().moe_set_dense_min_tokens(ctypes.c_void_p(h) if h else None, int(min_tokens)),
            "moe_set_dense_min_tokens")
+
+
+def moe_last_launches(h):
+    """Kernels launched by the handle's last moe_forward (see include/moe.h)."""
+    n = ctypes.c_int(0)
+    _check(_lib().moe_last_launches(ctypes.c_void_p(h) if h else None, ctypes.byref(n)),
+           "moe_last_launches")
+    return n.value
 
 
 def moe_destroy(h):

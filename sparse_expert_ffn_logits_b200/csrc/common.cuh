@@ -18,6 +18,12 @@ constexpr int kMaxTokens = 1024;
 constexpr int kMaxHsplit = 16;     // router slices of H
 constexpr int kMaxI = 16384;       // largest intermediate size
 
+// Per-pair histogram of the selection scores, filled by the gate epilogues and read by the
+// selection: bin = the top 12 bits of the score's fp32 pattern (its sign bit is 0), i.e. the
+// exponent and the 3 leading mantissa bits.  The 20 bits below are five 4-bit radix digits.
+constexpr int kHistBins = 2048;
+constexpr int kHistShift = 20;
+
 // device error word codes
 constexpr int kErrNanLogit = 1;
 constexpr int kErrNanAct = 2;
@@ -96,6 +102,11 @@ struct FwdParams {
   const void* zero_row;  // H zero elements (source of the copies of absent tokens)
   unsigned long long* trace;  // per-CTA phase timestamps (nullptr: tracing off)
   unsigned* claim;            // [2] work-item counters of the gate and up/down kernels
+  unsigned* hist;             // [Pmax][kHistBins] score histograms of top-K pairs (zero at rest)
+  // roster routing (nullptr: off): the router picks the top-k of logits + router_bias and adds
+  // its choice to roster_counts; the weights stay those of the unbiased logits
+  const float* router_bias;   // [B][E]
+  int* roster_counts;         // [B][E] per-sequence selection counts (the caller's)
   // dense masked fallback: a slot with T >= dense_min tokens is computed by the tcgen05 GEMMs
   int dense_min;              // INT_MAX: never
   int imax_pad;               // Imax rounded up to 128 (row length of hbuf)
@@ -231,6 +242,28 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* to
 }
 
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
+
+// Selection key of an activation: the fp32 pattern of |a|, which orders like the score; a NaN
+// activation scores 0.
+__device__ __forceinline__ uint32_t score_key(float a) {
+  return isnan(a) ? 0u : __float_as_uint(fabsf(a));
+}
+
+__device__ __forceinline__ void red_add_u32(unsigned* p, unsigned v) {
+  asm volatile("red.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Whether the pairs of kind (0 routed, 1 shared) are cut by the top-K radix selection, which
+// reads the score histogram (threshold mode, K = 0 and K = I need none).
+__device__ __forceinline__ bool uses_hist(const FwdParams& p, int kind) {
+  const int I = kind ? p.Ish : p.I;
+  return p.hist && p.sel_mode[kind] == 0 && p.sel_K[kind] > 0 && p.sel_K[kind] < I;
+}
+
+// Counts activation a of pair q in the pair's score histogram.
+__device__ __forceinline__ void hist_add(const FwdParams& p, int q, float a) {
+  red_add_u32(&p.hist[(size_t)q * kHistBins + (score_key(a) >> kHistShift)], 1u);
+}
 
 __device__ __forceinline__ void set_error(int* err, int code) { atomicCAS(err, 0, code); }
 

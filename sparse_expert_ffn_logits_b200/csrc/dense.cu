@@ -307,12 +307,14 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
         const int nc = min(32, r.ntok - c0);
         if (kMode == 0) {
           if (row < r.mext) {
+            const bool hist = uses_hist(p, r.kind);
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
               if (c < nc) {
                 const float a = silu(__uint_as_float(v[c]));
                 nan_seen |= isnan(a);
                 p.act[(size_t)(r.q0 + r.n0 + c0 + c) * p.Imax + row] = a;
+                if (hist) hist_add(p, r.q0 + r.n0 + c0 + c, a);
               }
             }
           }

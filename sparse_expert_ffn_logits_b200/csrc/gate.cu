@@ -324,6 +324,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, 
         const float a = silu(v);
         nan_seen |= isnan(a);
         p.act[(size_t)(q0 + ti) * p.Imax + n0 + (ln >> 2) + (c >> 1) * 8] = a;
+        if (uses_hist(p, q0 >= p.B * p.k)) hist_add(p, q0 + ti, a);
       }
     }
     if (mi == 0) trace_point(p.trace, 1, 4);
@@ -377,6 +378,7 @@ __global__ void __launch_bounds__(kThreads) gate_f32_kernel(FwdParams p) {
           const float a = silu(d[c]);
           nan_seen |= isnan(a);
           p.act[(size_t)(q0 + ti) * Imax + n0 + g + (c >> 1) * 8] = a;
+          if (uses_hist(p, kind)) hist_add(p, q0 + ti, a);
         }
       }
     }

@@ -37,6 +37,40 @@ __global__ void finalize_kernel(FwdParams p) {
   }
 }
 
+// Roster routing bias ("Predatory MoE", technical summary, Methodology 2): one CTA per sequence
+// t.  The roster is the m experts with the most selections so far (equal counts: lower index),
+// found by each expert's rank among the counts.  bias[t][e] = 0 while fewer than m distinct
+// experts have been used; then +delta for roster members and -delta for the others; for a
+// pinned sequence 0 for members and -inf for the others.
+__global__ void roster_bias_kernel(const int* __restrict__ counts, const int* __restrict__ pinned,
+                                   int E, int m, float delta, float* __restrict__ bias) {
+  __shared__ int c[kMaxRouted];
+  __shared__ int s_distinct;
+  const int t = blockIdx.x;
+  if (threadIdx.x == 0) s_distinct = 0;
+  __syncthreads();
+  int mine = 0;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    c[e] = counts[(size_t)t * E + e];
+    mine += c[e] > 0;
+  }
+  if (mine) atomicAdd(&s_distinct, mine);
+  __syncthreads();
+  const bool pin = pinned[t] != 0;
+  const bool explore = s_distinct < m;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int ce = c[e];
+    int rank = 0;
+    for (int f = 0; f < E; ++f) rank += c[f] > ce || (c[f] == ce && f < e);
+    const bool member = rank < m;
+    float b;
+    if (pin) b = member ? 0.f : -INFINITY;
+    else if (explore) b = 0.f;
+    else b = member ? delta : -delta;
+    bias[(size_t)t * E + e] = b;
+  }
+}
+
 // packed[e][n][1][h] = w_down[e][h][n]: 32x32 tiles through shared memory.
 template <typename T>
 __global__ void pack_down_kernel(const T* __restrict__ wd, T* __restrict__ ud, int I, int H) {
@@ -139,6 +173,12 @@ __global__ void force_timeout_kernel(FwdParams p) {
   __syncwarp();
   volatile int* abort = &s_abort;
   if (threadIdx.x == 0) mbar_wait(&bar, 0, abort, p.err);  // phase 0 never completes
+}
+
+cudaError_t launch_roster_bias(const int* counts, const int* pinned, int B, int E, int m,
+                               float delta, float* bias, cudaStream_t st) {
+  roster_bias_kernel<<<B, 128, 0, st>>>(counts, pinned, E, m, delta, bias);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_force_timeout(const FwdParams& p, cudaStream_t st) {

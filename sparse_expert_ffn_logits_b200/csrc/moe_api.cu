@@ -40,10 +40,12 @@ struct moe_handle {
   void* out_stage;
   bool dirty;       // a call failed mid-way: re-zero before the next one
   int last_tokens;
+  int last_launches;  // kernels the last moe_forward launched
   cudaEvent_t stage_events[MOE_STAGE_EVENTS];
   bool timing;
   int dense_min;  // MOE_DENSE_AUTO, 0 (never dense) or a per-slot token threshold
   unsigned long long* trace_buf;  // device, kTraceKernels * kTraceCtas * kTracePoints stamps
+  float* roster_bias;  // device [max_tokens][E]: the roster bias of the current call
 };
 
 namespace {
@@ -156,6 +158,7 @@ size_t carve(moe_handle* h, char* base) {
   p.ulist = cv.take<int>(slots * Im);
   p.ucnt = cv.take<int>(slots);
   p.err = cv.take<int>(1);
+  h->roster_bias = cv.take<float>(Bm * E);
   p.zero_row = cv.take<char>((size_t)c.hidden * h->elt);
   h->trace_buf = cv.take<unsigned long long>((size_t)moe::kTraceKernels * moe::kTraceCtas *
                                              moe::kTracePoints);
@@ -167,13 +170,14 @@ size_t carve(moe_handle* h, char* base) {
   const bool dense_ok = c.dtype == MOE_BF16;
   p.xp = dense_ok ? cv.take<__nv_bfloat16>(Pm * c.hidden) : nullptr;
   p.hbuf = dense_ok ? cv.take<__nv_bfloat16>(Pm * (size_t)p.imax_pad) : nullptr;
-  // zero-at-rest region: tickets, union bitmasks, output accumulator
+  // zero-at-rest region: tickets, union bitmasks, score histograms, output accumulator
   char* zb = cv.take<char>(0);
   p.tile_ticket = cv.take<unsigned>((Bm + moe::kTileTok - 1) / moe::kTileTok);
   p.global_ticket = cv.take<unsigned>(1);
   p.claim = cv.take<unsigned>(2);
   p.slot_ticket = cv.take<unsigned>(slots);
   p.ubits = cv.take<uint32_t>(slots * Wm);
+  p.hist = cv.take<unsigned>(Pm * moe::kHistBins);
   p.out_acc = cv.take<float>(Bm * c.hidden);
   h->zero_begin = zb;
   h->zero_bytes = (size_t)((base + cv.off) - zb);
@@ -183,9 +187,9 @@ size_t carve(moe_handle* h, char* base) {
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 moe_status forward_impl(moe_handle* h, const void* x, int n_tokens, const void* router,
-                        const moe_expert_weights* routed, const moe_expert_weights* shared,
-                        const moe_sparsity* sp_routed, const moe_sparsity* sp_shared, void* out,
-                        cudaStream_t st) {
+                        const moe_roster* roster, const moe_expert_weights* routed,
+                        const moe_expert_weights* shared, const moe_sparsity* sp_routed,
+                        const moe_sparsity* sp_shared, void* out, cudaStream_t st) {
   const moe_config& c = h->cfg;
   FwdParams p = h->base;
   p.H = c.hidden;
@@ -238,6 +242,15 @@ moe_status forward_impl(moe_handle* h, const void* x, int n_tokens, const void* 
   const bool dense = p.dense_min <= n_tokens;
   cudaEvent_t* ev = h->stage_events;
   cudaError_t e = tm ? cudaEventRecord(ev[0], st) : cudaSuccess;
+  p.router_bias = nullptr;
+  p.roster_counts = nullptr;
+  if (roster) {
+    p.router_bias = h->roster_bias;
+    p.roster_counts = roster->counts;
+    if (e == cudaSuccess)
+      e = moe::launch_roster_bias(roster->counts, roster->pinned, n_tokens, c.n_routed, roster->m,
+                                  roster->delta, h->roster_bias, st);
+  }
   if (e == cudaSuccess) e = moe::launch_router(p, dt, st);
   if (e == cudaSuccess && tm) e = cudaEventRecord(ev[1], st);
   if (e == cudaSuccess) e = moe::launch_gate(p, dt, h->ls, st, pdl);
@@ -255,6 +268,8 @@ moe_status forward_impl(moe_handle* h, const void* x, int n_tokens, const void* 
     return MOE_ERR_CUDA;
   }
   h->last_tokens = n_tokens;
+  // + gather and three GEMMs on the tensor-core path, + the roster bias kernel
+  h->last_launches = (dense ? 9 : 5) + (roster ? 1 : 0);
   return MOE_OK;
 }
 
@@ -371,7 +386,27 @@ moe_status moe_forward(moe_handle* h, const void* x, int n_tokens, const void* r
   if (n_tokens == 0) return MOE_OK;
   DeviceScope dev(h->device);
   if (!dev.ok) return MOE_ERR_CUDA;
-  return forward_impl(h, x, n_tokens, router, routed, shared, sp_routed, sp_shared, out,
+  return forward_impl(h, x, n_tokens, router, nullptr, routed, shared, sp_routed, sp_shared, out,
+                      static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_forward_roster(moe_handle* h, const void* x, int n_tokens, const void* router,
+                              const moe_roster* roster, const moe_expert_weights* routed,
+                              const moe_expert_weights* shared, const moe_sparsity* sp_routed,
+                              const moe_sparsity* sp_shared, void* out, void* stream) {
+  moe_status s = check_forward(h, x, n_tokens, router, routed, shared, sp_routed, sp_shared, out,
+                               false);
+  if (s != MOE_OK) return s;
+  if (n_tokens == 0) return MOE_OK;
+  if (!roster || !roster->counts || !roster->pinned) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(roster->counts) | reinterpret_cast<uintptr_t>(roster->pinned)) &
+      3u)
+    return MOE_ERR_INVALID_ARG;
+  if (roster->m < h->cfg.top_k || roster->m > h->cfg.n_routed) return MOE_ERR_INVALID_ARG;
+  if (!(roster->delta >= 0.f) || isinf(roster->delta)) return MOE_ERR_INVALID_ARG;
+  DeviceScope dev(h->device);
+  if (!dev.ok) return MOE_ERR_CUDA;
+  return forward_impl(h, x, n_tokens, router, roster, routed, shared, sp_routed, sp_shared, out,
                       static_cast<cudaStream_t>(stream));
 }
 
@@ -389,7 +424,7 @@ moe_status moe_forward_host(moe_handle* h, const void* x_host, int n_tokens, con
   const size_t bytes = (size_t)n_tokens * h->cfg.hidden * h->elt;
   if (cudaMemcpyAsync(h->x_stage, x_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
     return MOE_ERR_CUDA;
-  s = forward_impl(h, h->x_stage, n_tokens, router, routed, shared, sp_routed, sp_shared,
+  s = forward_impl(h, h->x_stage, n_tokens, router, nullptr, routed, shared, sp_routed, sp_shared,
                    h->out_stage, st);
   if (s != MOE_OK) return s;
   if (cudaMemcpyAsync(out_host, h->out_stage, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
@@ -472,6 +507,12 @@ moe_status moe_debug_force_timeout(moe_handle* h, void* stream) {
   DeviceScope dev(h->device);
   if (!dev.ok) return MOE_ERR_CUDA;
   return cuda_status(moe::launch_force_timeout(h->base, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_last_launches(moe_handle* h, int* n) {
+  if (!h || !n) return MOE_ERR_INVALID_ARG;
+  *n = h->last_launches;
+  return MOE_OK;
 }
 
 moe_status moe_set_dense_min_tokens(moe_handle* h, int min_tokens) {

@@ -34,13 +34,17 @@ __device__ __forceinline__ float key_value(unsigned long long k) {
 }
 
 // Top-k of one token's logits (lg, shared memory) by one warp; writes topk_idx / topk_w.
-// PER = logits per lane (E <= 32 * PER).  sv / si: this warp's k-entry scratch.
+// PER = logits per lane (E <= 32 * PER).  sv / si: this warp's k-entry scratch.  With roster
+// routing the choice is by logit + bias (the bias row of the token's sequence), the weights come
+// from the unbiased logits, and the sequence's counts of the chosen experts grow by one.
 template <int PER>
 __device__ void topk_token(const FwdParams& p, int tok, const float* lg, float* sv, int* si) {
   const int lane = threadIdx.x & 31;
   const int E = p.E, k = p.k;
+  const float* bias = p.router_bias ? p.router_bias + (size_t)tok * E : nullptr;
   unsigned long long key[PER];
   bool nan_seen = false;
+  float mx = -INFINITY;  // largest unbiased logit (the softmax-over-all shift)
 #pragma unroll
   for (int j = 0; j < PER; ++j) {
     const int e = lane + 32 * j;
@@ -51,6 +55,9 @@ __device__ void topk_token(const FwdParams& p, int tok, const float* lg, float* 
         nan_seen = true;
         f = -INFINITY;
       }
+      mx = fmaxf(mx, f);
+      if (bias) f = f + __ldg(bias + e);
+      if (isnan(f)) f = -INFINITY;
       key[j] = topk_key(f, e);
     }
   }
@@ -70,13 +77,25 @@ __device__ void topk_token(const FwdParams& p, int tok, const float* lg, float* 
       if (lane + 32 * j == e) key[j] = 0ull;
     if (lane == 0) {
       si[r] = e;
-      sv[r] = key_value(best);
+      const float f = lg[e];
+      sv[r] = isnan(f) ? -INFINITY : f;  // the unbiased logit of the chosen expert
     }
   }
   __syncwarp();
-  // routing weights: lane r < k computes entry r
+  // routing weights: lane r < k computes entry r.  The shift is the largest chosen logit
+  // (softmax over the chosen) or the largest logit (softmax over all); without a bias both are
+  // the first chosen logit.
   float z = 0.f;
-  const float m = sv[0];
+  float m = sv[0];
+  if (bias) {
+    if (p.route == 1) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      m = mx;
+    } else {
+      for (int r = 1; r < k; ++r) m = fmaxf(m, sv[r]);
+    }
+  }
   if (p.route == 1) {
 #pragma unroll
     for (int j = 0; j < PER; ++j) {
@@ -96,6 +115,7 @@ __device__ void topk_token(const FwdParams& p, int tok, const float* lg, float* 
     const float w = p.route == 2 ? 1.0f / (1.0f + expf(-v)) : expf(v - m) / z;
     p.topk_idx[(size_t)tok * k + lane] = si[lane];
     p.topk_w[(size_t)tok * k + lane] = w;
+    if (p.roster_counts) p.roster_counts[(size_t)tok * E + si[lane]] += 1;
   }
 }
 

@@ -92,6 +92,43 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
       // most 32 keys share the prefix, one warp ranks them directly.
       uint32_t prefix = 0, pmask = 0;
       int krem = K, cand = I, shift = 28, pass = 0;
+      if (uses_hist(p, kind)) {
+        // The gate counted this pair's keys by their top 12 bits.  Thread r owns the 8 bins
+        // counted from the top, [8 (255 - r), 8 (256 - r)); an exclusive scan in thread order
+        // gives the keys in the bins above them, and the thread whose bins hold the K-th largest
+        // key names its bin.  The row is cleared for the next call.
+        static_assert(kHistBins == 8 * kSelThreads, "8 histogram bins per thread");
+        unsigned* hrow = p.hist + (size_t)q * kHistBins;
+        const int b0 = 8 * (kSelThreads - 1 - threadIdx.x);
+        const uint4 h0 = __ldcg(reinterpret_cast<const uint4*>(hrow + b0));
+        const uint4 h1 = __ldcg(reinterpret_cast<const uint4*>(hrow + b0 + 4));
+        *reinterpret_cast<uint4*>(hrow + b0) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(hrow + b0 + 4) = make_uint4(0, 0, 0, 0);
+        const unsigned hb[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+        int mine = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mine += (int)hb[i];
+        int above = block_exclusive_scan(mine, reinterpret_cast<int*>(hist), nullptr);
+        if (above < K && above + mine >= K) {
+#pragma unroll
+          for (int i = 7; i >= 0; --i) {
+            const int c = (int)hb[i];
+            if (above < K && above + c >= K) {
+              s_tau = (uint32_t)(b0 + i);
+              s_need = K - above;
+              s_eqtot = c;
+            }
+            above += c;
+          }
+        }
+        __syncthreads();
+        prefix = s_tau << kHistShift;
+        pmask = ~0u << kHistShift;
+        krem = s_need;
+        cand = s_eqtot;
+        shift = kHistShift - 4;
+        __syncthreads();  // s_tau and friends are written again below
+      }
 #pragma unroll 1
       for (; shift >= 0 && cand > 32; shift -= 4, ++pass) {
         uint32_t c[8] = {0, 0, 0, 0, 0, 0, 0, 0};

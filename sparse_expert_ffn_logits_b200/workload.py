@@ -9,7 +9,8 @@ import torch
 import synth
 
 from . import (expert_weights, make_config, moe_create, moe_debug_lists, moe_destroy,
-               moe_forward, moe_pack_experts, sparsity)
+               moe_forward, moe_forward_roster, moe_last_launches, moe_pack_experts, roster,
+               sparsity)
 
 
 class DeviceLayer:
@@ -33,6 +34,7 @@ class DeviceLayer:
             self.shared = expert_weights(self.sh_gate, self.sh_updown)
         else:
             self.shared = None
+        self.roster = None  # (counts, pinned, m, delta): calls use roster routing when set
         torch.cuda.synchronize()
 
     def _pack(self, shared, n, I, chunk, device):
@@ -64,12 +66,22 @@ class DeviceLayer:
             out = torch.empty_like(x)
         sr = sparsity(rule_routed)
         ss = sparsity(rule_shared) if (self.shape.n_shared and rule_shared) else None
-        moe_forward(self.h, x, x.shape[0], self.router, self.routed, self.shared, sr, ss, out,
-                    stream)
+        if self.roster is not None:
+            counts, pinned, m, delta = self.roster
+            moe_forward_roster(self.h, x, x.shape[0], self.router,
+                               roster(counts, pinned, m, delta), self.routed, self.shared, sr, ss,
+                               out, stream)
+        else:
+            moe_forward(self.h, x, x.shape[0], self.router, self.routed, self.shared, sr, ss,
+                        out, stream)
         return out
 
     def debug(self, n_tokens):
-        """Intermediate results of the last call: idx, w, logits, cnt, lists, act."""
+        """Intermediate results of the last call: idx, w, logits, cnt, lists, act (numpy)."""
+        return {k: v.cpu().numpy() for k, v in self.debug_device(n_tokens).items()}
+
+    def debug_device(self, n_tokens):
+        """The same as debug(), as tensors on the layer's device."""
         s = self.shape
         P = s.top_k + s.n_shared
         imax = max(s.inter, s.inter_shared if s.n_shared else 0)
@@ -83,7 +95,10 @@ class DeviceLayer:
         moe_debug_lists(self.h, n_tokens, r["idx"], r["w"], r["logits"], r["cnt"], r["lists"],
                         r["act"])
         torch.cuda.synchronize()
-        return {k: v.cpu().numpy() for k, v in r.items()}
+        return r
+
+    def last_launches(self):
+        return moe_last_launches(self.h)
 
     def close(self):
         if self.h:

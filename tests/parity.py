@@ -99,11 +99,15 @@ def _classify(gap, cut, bound):
 
 
 def compare(dl, x_host, x_dev, rule_r, rule_s=None, tokens=None, shared_weights=None,
-            expert_cache=None, router_host=None, allow_fp32_bound=0, name=None):
+            expert_cache=None, router_host=None, allow_fp32_bound=0, name=None,
+            router_bias=None):
     """Runs the layer on x_dev and checks it against the oracle on x_host (same values).
     Routing and selection are checked for every token; ``tokens`` restricts only the output
     comparison to a subset of tokens (sampled check).  ``allow_fp32_bound`` is the number of
-    fp32-bound-only exemptions this comparison may take (0: any fails it)."""
+    fp32-bound-only exemptions this comparison may take (0: any fails it).  ``router_bias``
+    ([B][E], the oracle's roster bias of this call, exact in fp32) makes the oracle choose the
+    top-k of logits + bias, as the layer does under roster routing.  The report's ``idx`` is the
+    routing the comparison adopted (the layer's)."""
     shape = dl.shape
     B = x_host.shape[0]
     k, S, I, Ish, H = shape.top_k, shape.n_shared, shape.inter, shape.inter_shared, shape.hidden
@@ -122,21 +126,27 @@ def compare(dl, x_host, x_dev, rule_r, rule_s=None, tokens=None, shared_weights=
 
     # ---- routing, every token
     rl = oracle.Layer(shape, router, {}, [])
-    logits_o, idx_o, _ = rl.route(x_host)
+    logits_o, idx_o, _ = rl.route_biased(x_host, router_bias)
+    bias32 = None if router_bias is None else np.asarray(router_bias, np.float32)
     idx_use = idx_o.copy()
     for t in range(B):
         rep.tokens_routed += 1
         g_idx = dbg["idx"][t]
-        # second check: the oracle's top-k on the GPU's own logits
-        assert np.array_equal(oracle.topk(dbg["logits"][t].astype(np.float64), k), g_idx), \
+        # second check: the oracle's top-k on the GPU's own logits (plus the bias, added in fp32
+        # as the layer adds it)
+        g_sel = dbg["logits"][t].astype(np.float32)
+        if bias32 is not None:
+            g_sel = g_sel + bias32[t]
+        assert np.array_equal(oracle.topk(g_sel.astype(np.float64), k), g_idx), \
             f"top-k logic differs on token {t}"
         idx_use[t] = g_idx
         if np.array_equal(np.sort(g_idx), np.sort(idx_o[t])):
             continue
-        lo = logits_o[t]
+        lo = logits_o[t] + (0.0 if router_bias is None else np.asarray(router_bias)[t])
         order = np.lexsort((np.arange(shape.n_routed), -lo))
         cut = lo[order[k - 1]]
-        bound = H * U32 * (np.abs(wr) @ np.abs(xf[t]))
+        # the fp32 logits, then the fp32 addition of the bias (one more rounding)
+        bound = H * U32 * (np.abs(wr) @ np.abs(xf[t])) + U32 * np.abs(lo)
         for e in set(g_idx.tolist()) ^ set(idx_o[t].tolist()):
             gap = abs(lo[e] - cut)
             b = bound[e] + bound[order[k - 1]]
@@ -230,6 +240,7 @@ def compare(dl, x_host, x_dev, rule_r, rule_s=None, tokens=None, shared_weights=
     scale = np.maximum(np.abs(r), np.sqrt(np.mean(r * r)) if r.size else 1.0)
     err = np.abs(g - r) / np.maximum(scale, 1e-30)
     rep.max_err = float(err.max()) if err.size else 0.0
+    rep.idx = idx_use
     RECORDS.append(rep)
     tol = tolerance(shape)
     assert rep.max_err <= tol, f"output error {rep.max_err:.3e} > {tol} ({rep})"

@@ -87,6 +87,13 @@ def test_forward_rejects_null_handle(lib):
         moe.MOE_ERR_INVALID_ARG
     assert lib.moe_set_dense_min_tokens(None, 8) == moe.MOE_ERR_INVALID_ARG
     assert lib.moe_debug_force_timeout(None, None) == moe.MOE_ERR_INVALID_ARG
+    n = ctypes.c_int(-1)
+    assert lib.moe_last_launches(None, ctypes.byref(n)) == moe.MOE_ERR_INVALID_ARG
+    ro = moe.MoERoster(16, 16, 4, 0.5)
+    rc = lib.moe_forward_roster(None, ctypes.c_void_p(16), 1, ctypes.c_void_p(16),
+                                ctypes.byref(ro), ctypes.byref(rw), None, ctypes.byref(sp), None,
+                                ctypes.c_void_p(16), None)
+    assert rc == moe.MOE_ERR_INVALID_ARG
 
 
 def test_status_strings(lib):
