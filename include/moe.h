@@ -226,6 +226,32 @@ moe_status moe_debug_force_timeout(moe_handle* h, void* stream);
 #define MOE_DENSE_AUTO (-1)
 moe_status moe_set_dense_min_tokens(moe_handle* h, int min_tokens);
 
+/* Expert parallelism ("Uncovering Intra-expert Activation Sparsity ...", technical summary,
+ * Methodology: the serving system keeps expert parallelism).  Each of G ranks holds a handle of
+ * the same configuration restricted to the routed experts [e_begin, e_end) and to the shared
+ * experts whose bit is set in shared_mask; together the ranks' ranges and masks cover every
+ * expert once.  Every handle still routes every token over all E experts (the router weights
+ * and the tokens are replicated), so the ranks agree on the routing.  A restricted handle reads
+ * routed weights of its own experts only: `routed` of its calls points at the packed blocks of
+ * experts e_begin .. e_end - 1 (expert e at local index e - e_begin); `shared` still points at
+ * all S shared experts' blocks, of which it reads the masked ones.  Default: all experts.
+ * INVALID_ARG for a NULL handle, a range outside [0, E] or a mask bit at or above S. */
+moe_status moe_set_expert_range(moe_handle* h, int e_begin, int e_end, unsigned shared_mask);
+
+/* moe_forward that writes this handle's part of the layer output in fp32 instead of the cast
+ * output: partial [n_tokens][H] (device, fp32, 16-byte aligned) = the weighted sum over the
+ * (token, expert) pairs of the handle's experts.  The sum of the ranks' partials (an
+ * all-reduce) is the layer output before rounding; moe_cast_output rounds it. */
+moe_status moe_forward_partial(moe_handle* h, const void* x, int n_tokens, const void* router,
+                               const moe_expert_weights* routed, const moe_expert_weights* shared,
+                               const moe_sparsity* sp_routed, const moe_sparsity* sp_shared,
+                               float* partial, void* stream);
+
+/* out [n_tokens][H] (cfg.dtype) = sum [n_tokens][H] (fp32) rounded to the layer dtype, on
+ * `stream`.  Both device buffers 16-byte aligned. */
+moe_status moe_cast_output(moe_handle* h, const float* sum, int n_tokens, void* out,
+                           void* stream);
+
 /* How many kernels the last successful moe_forward on this handle launched (5 on the sparse
  * path: router, gate, select, up/down, output cast; 9 when the tensor-core path ran as well;
  * one more with roster routing; 0 before the first call).  Host-side only: reads no device memory.  INVALID_ARG for NULL. */

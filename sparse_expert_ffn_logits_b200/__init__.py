@@ -58,7 +58,8 @@ EXPORTS = ("moe_create", "moe_packed_bytes", "moe_pack_experts", "moe_forward",
            "moe_forward_roster",
            "moe_forward_host", "moe_debug_lists", "moe_profile_stages", "moe_read_trace",
            "moe_get_error", "moe_debug_force_timeout", "moe_set_dense_min_tokens",
-           "moe_last_launches", "moe_destroy",
+           "moe_last_launches", "moe_set_expert_range", "moe_forward_partial",
+           "moe_cast_output", "moe_destroy",
            "moe_route_noalloc",
            "moe_status_string")
 MOE_STAGE_EVENTS = 6
@@ -94,6 +95,9 @@ def _lib():
         lib.moe_destroy.argtypes = [P]
         lib.moe_set_dense_min_tokens.argtypes = [P, I]
         lib.moe_last_launches.argtypes = [P, ctypes.POINTER(I)]
+        lib.moe_set_expert_range.argtypes = [P, I, I, ctypes.c_uint]
+        lib.moe_forward_partial.argtypes = fwd
+        lib.moe_cast_output.argtypes = [P, P, I, P, P]
         lib.moe_debug_force_timeout.argtypes = [P, P]
         lib.moe_route_noalloc.argtypes = [ctypes.POINTER(MoEConfig), P, I, P, P, P, P]
         lib.moe_status_string.argtypes = [I]
@@ -260,6 +264,27 @@ def moe_last_launches(h):
     _check(_lib().moe_last_launches(ctypes.c_void_p(h) if h else None, ctypes.byref(n)),
            "moe_last_launches")
     return n.value
+
+
+def moe_set_expert_range(h, e_begin, e_end, shared_mask):
+    """Restricts the handle to routed experts [e_begin, e_end) and the masked shared experts."""
+    _check(_lib().moe_set_expert_range(ctypes.c_void_p(h) if h else None, int(e_begin),
+                                       int(e_end), int(shared_mask)), "moe_set_expert_range")
+
+
+def moe_forward_partial(h, x, n_tokens, router, routed, shared, sp_routed, sp_shared, partial,
+                        stream=None):
+    _check(_lib().moe_forward_partial(ctypes.c_void_p(h), _ptr(x), int(n_tokens), _ptr(router),
+                                      ctypes.byref(routed),
+                                      ctypes.byref(shared) if shared else None,
+                                      ctypes.byref(sp_routed),
+                                      ctypes.byref(sp_shared) if sp_shared else None,
+                                      _ptr(partial), _stream(stream)), "moe_forward_partial")
+
+
+def moe_cast_output(h, partial_sum, n_tokens, out, stream=None):
+    _check(_lib().moe_cast_output(ctypes.c_void_p(h), _ptr(partial_sum), int(n_tokens), _ptr(out),
+                                  _stream(stream)), "moe_cast_output")
 
 
 def moe_destroy(h):

@@ -66,6 +66,8 @@ struct FwdParams {
   int H, E, k, S, I, Ish, B, Imax;
   int Bmax;         // max_tokens of the handle
   int hsplit;       // router slices of H
+  int e_begin, e_end;     // routed experts this handle evaluates (expert parallelism)
+  unsigned shared_mask;   // shared experts this handle evaluates (bit s = shared expert s)
   int router_cluster;  // CTAs of the single-cluster router on this device (0: multi-CTA only)
   int route;
   int sel_mode[2];  // [0] routed, [1] shared: 0 top-K, 1 threshold

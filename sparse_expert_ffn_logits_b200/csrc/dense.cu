@@ -372,7 +372,7 @@ __global__ void gather_kernel(FwdParams p) {
   const int w0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, nw = (gridDim.x * blockDim.x) >> 5;
   for (int q = w0; q < n_pairs; q += nw) {
     const int j = __ldcg(&p.pair_slot[q]);
-    if (!slot_is_dense(__ldcg(&p.slots[j].T), p.dense_min)) continue;
+    if (j < 0 || !slot_is_dense(__ldcg(&p.slots[j].T), p.dense_min)) continue;
     const int tok = __ldcg(&p.pair_token[q]);
     const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(p.x) + (size_t)tok * p.H;
     for (int v = lane; v < p.H / 8; v += 32)
@@ -430,7 +430,8 @@ cudaError_t configure_dense(int budget) {
 cudaError_t launch_dense(const FwdParams& p, const LaunchShape& ls, int stage, cudaStream_t st,
                          bool pdl) {
   const uint64_t H = (uint64_t)p.H;
-  const uint64_t rows_r = (uint64_t)p.E * p.I, rows_s = (uint64_t)p.S * p.Ish;
+  // the routed weights are the handle's local block of experts [e_begin, e_end)
+  const uint64_t rows_r = (uint64_t)(p.e_end - p.e_begin) * p.I, rows_s = (uint64_t)p.S * p.Ish;
   const __nv_bfloat16* gr = static_cast<const __nv_bfloat16*>(p.gate_r);
   const __nv_bfloat16* gs = static_cast<const __nv_bfloat16*>(p.gate_s);
   const __nv_bfloat16* ur = static_cast<const __nv_bfloat16*>(p.updown_r);

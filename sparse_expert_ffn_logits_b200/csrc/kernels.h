@@ -58,6 +58,8 @@ size_t select_smem_bytes(int imax);
 cudaError_t launch_pack_down(const void* w_down, void* packed_updown, int n, int I, int H,
                              int elt, cudaStream_t st);
 cudaError_t launch_force_timeout(const FwdParams& p, cudaStream_t st);
+cudaError_t launch_cast_output(const float* sum, void* out, size_t n, int dtype, int nsm,
+                               cudaStream_t st);
 cudaError_t launch_roster_bias(const int* counts, const int* pinned, int B, int E, int m,
                                float delta, float* bias, cudaStream_t st);
 cudaError_t launch_debug_gather(const FwdParams& p, int n_tokens, int* cnt, int* lists,

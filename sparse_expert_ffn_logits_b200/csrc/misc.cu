@@ -71,6 +71,24 @@ __global__ void roster_bias_kernel(const int* __restrict__ counts, const int* __
   }
 }
 
+// out[i] = dtype(sum[i]): the layer output from the sum of the partial outputs of all handles
+// (expert parallelism).
+template <typename T>
+__global__ void cast_output_kernel(const float* __restrict__ sum, T* __restrict__ out, size_t n4) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const float4 v = reinterpret_cast<const float4*>(sum)[i];
+    if constexpr (sizeof(T) == 2) {
+      uint2 o;
+      o.x = pack_bf16x2(v.x, v.y);
+      o.y = pack_bf16x2(v.z, v.w);
+      reinterpret_cast<uint2*>(out)[i] = o;
+    } else {
+      reinterpret_cast<float4*>(out)[i] = v;
+    }
+  }
+}
+
 // packed[e][n][1][h] = w_down[e][h][n]: 32x32 tiles through shared memory.
 template <typename T>
 __global__ void pack_down_kernel(const T* __restrict__ wd, T* __restrict__ ud, int I, int H) {
@@ -100,6 +118,14 @@ __global__ void debug_gather_kernel(FwdParams p, int* cnt, int* lists, float* ac
   const int q = p.pair_index[t * P + jj];
   const int I = jj < p.k ? p.I : p.Ish;
   const int lane = threadIdx.x & 31;
+  if (q < 0) {  // an expert another handle evaluates: no kept neuron, no activation here
+    for (int n = threadIdx.x; n < p.Imax; n += blockDim.x) {
+      if (lists) lists[(size_t)tj * p.Imax + n] = -1;
+      if (act) act[(size_t)tj * p.Imax + n] = 0.f;
+    }
+    if (threadIdx.x == 0 && cnt) cnt[tj] = 0;
+    return;
+  }
   const uint32_t* mrow = p.maskbits + (size_t)q * (p.Imax / 32);
   if (threadIdx.x < 32) {
     const int W = I / 32, wpl = (W + 31) / 32;
@@ -173,6 +199,20 @@ __global__ void force_timeout_kernel(FwdParams p) {
   __syncwarp();
   volatile int* abort = &s_abort;
   if (threadIdx.x == 0) mbar_wait(&bar, 0, abort, p.err);  // phase 0 never completes
+}
+
+cudaError_t launch_cast_output(const float* sum, void* out, size_t n, int dtype, int nsm,
+                               cudaStream_t st) {
+  const size_t n4 = n / 4;
+  size_t blocks = (n4 + 255) / 256;
+  if (blocks > (size_t)nsm * 4) blocks = (size_t)nsm * 4;
+  if (blocks == 0) return cudaSuccess;
+  if (dtype == 0)
+    cast_output_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
+        sum, static_cast<__nv_bfloat16*>(out), n4);
+  else
+    cast_output_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(sum, static_cast<float*>(out), n4);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_roster_bias(const int* counts, const int* pinned, int B, int E, int m,

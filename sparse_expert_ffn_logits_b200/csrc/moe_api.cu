@@ -46,6 +46,8 @@ struct moe_handle {
   int dense_min;  // MOE_DENSE_AUTO, 0 (never dense) or a per-slot token threshold
   unsigned long long* trace_buf;  // device, kTraceKernels * kTraceCtas * kTracePoints stamps
   float* roster_bias;  // device [max_tokens][E]: the roster bias of the current call
+  int e_begin, e_end;     // routed experts this handle evaluates (all by default)
+  unsigned shared_mask;   // shared experts this handle evaluates (all by default)
 };
 
 namespace {
@@ -189,7 +191,8 @@ moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_E
 moe_status forward_impl(moe_handle* h, const void* x, int n_tokens, const void* router,
                         const moe_roster* roster, const moe_expert_weights* routed,
                         const moe_expert_weights* shared, const moe_sparsity* sp_routed,
-                        const moe_sparsity* sp_shared, void* out, cudaStream_t st) {
+                        const moe_sparsity* sp_shared, void* out, cudaStream_t st,
+                        bool partial = false) {
   const moe_config& c = h->cfg;
   FwdParams p = h->base;
   p.H = c.hidden;
@@ -203,6 +206,9 @@ moe_status forward_impl(moe_handle* h, const void* x, int n_tokens, const void* 
   p.Bmax = c.max_tokens;
   p.hsplit = moe::router_hsplit(c.n_routed, n_tokens, c.hidden);
   p.router_cluster = h->ls.router_cluster;
+  p.e_begin = h->e_begin;
+  p.e_end = h->e_end;
+  p.shared_mask = h->shared_mask;
   p.route = (int)c.route;
   p.sel_mode[0] = sp_routed->mode == MOE_SEL_THRESHOLD ? 1 : 0;
   p.sel_K[0] = keep_count(c.inter, sp_routed->sparsity);
@@ -261,7 +267,8 @@ moe_status forward_impl(moe_handle* h, const void* x, int n_tokens, const void* 
   if (e == cudaSuccess && dense) e = moe::launch_dense(p, h->ls, 1, st, pdl);
   if (e == cudaSuccess) e = moe::launch_updown(p, dt, h->ls, st, pdl);
   if (e == cudaSuccess && tm) e = cudaEventRecord(ev[4], st);
-  if (e == cudaSuccess) e = moe::launch_finalize(p, dt, h->ls, st, pdl);
+  // a partial output stays fp32: the sum over the handles is cast once (moe_cast_output)
+  if (e == cudaSuccess) e = moe::launch_finalize(p, partial ? 1 : dt, h->ls, st, pdl);
   if (e == cudaSuccess && tm) e = cudaEventRecord(ev[5], st);
   if (e != cudaSuccess) {
     h->dirty = true;
@@ -331,6 +338,9 @@ moe_status moe_create(const moe_config* cfg, moe_handle** out) {
     return MOE_ERR_OOM;
   }
   h->dense_min = MOE_DENSE_AUTO;
+  h->e_begin = 0;
+  h->e_end = cfg->n_routed;
+  h->shared_mask = (1u << cfg->n_shared) - 1u;
   carve(h, static_cast<char*>(h->ws));
   if (cudaMemset(h->ws, 0, h->ws_bytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
     cudaFree(h->ws);
@@ -507,6 +517,41 @@ moe_status moe_debug_force_timeout(moe_handle* h, void* stream) {
   DeviceScope dev(h->device);
   if (!dev.ok) return MOE_ERR_CUDA;
   return cuda_status(moe::launch_force_timeout(h->base, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_set_expert_range(moe_handle* h, int e_begin, int e_end, unsigned shared_mask) {
+  if (!h || e_begin < 0 || e_end > h->cfg.n_routed || e_begin > e_end) return MOE_ERR_INVALID_ARG;
+  if (h->cfg.n_shared < 32 && (shared_mask >> h->cfg.n_shared) != 0u) return MOE_ERR_INVALID_ARG;
+  h->e_begin = e_begin;
+  h->e_end = e_end;
+  h->shared_mask = shared_mask;
+  return MOE_OK;
+}
+
+moe_status moe_forward_partial(moe_handle* h, const void* x, int n_tokens, const void* router,
+                               const moe_expert_weights* routed, const moe_expert_weights* shared,
+                               const moe_sparsity* sp_routed, const moe_sparsity* sp_shared,
+                               float* partial, void* stream) {
+  moe_status s = check_forward(h, x, n_tokens, router, routed, shared, sp_routed, sp_shared,
+                               partial, false);
+  if (s != MOE_OK) return s;
+  if (n_tokens == 0) return MOE_OK;
+  DeviceScope dev(h->device);
+  if (!dev.ok) return MOE_ERR_CUDA;
+  return forward_impl(h, x, n_tokens, router, nullptr, routed, shared, sp_routed, sp_shared,
+                      partial, static_cast<cudaStream_t>(stream), true);
+}
+
+moe_status moe_cast_output(moe_handle* h, const float* sum, int n_tokens, void* out,
+                           void* stream) {
+  if (!h || n_tokens < 0 || n_tokens > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+  if (n_tokens == 0) return MOE_OK;
+  if (!sum || !out || !aligned16(sum) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  DeviceScope dev(h->device);
+  if (!dev.ok) return MOE_ERR_CUDA;
+  return cuda_status(moe::launch_cast_output(sum, out, (size_t)n_tokens * h->cfg.hidden,
+                                             h->cfg.dtype == MOE_BF16 ? 0 : 1, h->ls.nsm,
+                                             static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_last_launches(moe_handle* h, int* n) {

@@ -150,6 +150,9 @@ extern "C" moe_status moe_route_noalloc(const moe_config* cfg, const void* x, in
   p.router_cluster = cluster;
   p.route = (int)cfg->route;
   p.dense_min = INT_MAX;  // only the grouping's item counts read it; no later kernel runs
+  p.e_begin = 0;
+  p.e_end = E;
+  p.shared_mask = 0;
   p.x = x;
   p.router = router;
   p.logits = reinterpret_cast<float*>(base + o_logits);

@@ -151,7 +151,10 @@ __device__ unsigned long long block_scan64(unsigned long long v, unsigned long l
 
 // Groups all pairs by expert (tokens ascending within an expert) and writes the slot table,
 // the pair arrays and meta (one CTA).  One 64-bit block scan over the experts gives, packed,
-// each expert's first pair, its slot index and its first gate item.
+// each expert's first pair, its slot index and its first gate item.  Under expert parallelism
+// only the routed experts [e_begin, e_end) and the shared experts of shared_mask are this
+// handle's: the others get no slot, their pairs no pair index (pair_slot -1), and a slot names
+// its routed expert by its index in the handle's local block of weights (e - e_begin).
 __device__ void group_pairs(const FwdParams& p, uint32_t* dyn, unsigned long long* scratch) {
   const int B = p.B, E = p.E, k = p.k, S = p.S;
   const int W = (B + 31) / 32;
@@ -174,41 +177,41 @@ __device__ void group_pairs(const FwdParams& p, uint32_t* dyn, unsigned long lon
     atomicOr(&tokmask[e * W + (t >> 5)], 1u << (t & 31));
   }
   __syncthreads();
-  // packed per expert: pairs (bits 0..19) | touched (bits 20..31) | gate items (bits 32..63)
-  const int per = (E + blockDim.x - 1) / blockDim.x;
-  const int e0 = min(E, (int)threadIdx.x * per), e1 = min(E, e0 + per);
-  unsigned long long mine = 0ull;
-  for (int e = e0; e < e1; ++e) {
+  // packed per local expert: pairs (bits 0..19) | touched (bits 20..31) | gate items (32..63)
+  auto packed = [&](int e) -> unsigned long long {
+    if (e < p.e_begin || e >= p.e_end) return 0ull;
     const unsigned long long c = (unsigned)cnt[e];
     // a dense slot (c >= dense_min) has no sparse gate items: the tensor-core path covers it
     const unsigned long long items =
         c && (int)c < p.dense_min
             ? (unsigned long long)(p.I / kTileRows) * ((c + kTileTok - 1) / kTileTok)
             : 0ull;
-    mine += c | ((c ? 1ull : 0ull) << 20) | (items << 32);
-  }
+    return c | ((c ? 1ull : 0ull) << 20) | (items << 32);
+  };
+  const int per = (E + blockDim.x - 1) / blockDim.x;
+  const int e0 = min(E, (int)threadIdx.x * per), e1 = min(E, e0 + per);
+  unsigned long long mine = 0ull;
+  for (int e = e0; e < e1; ++e) mine += packed(e);
   unsigned long long tot;
   unsigned long long run = block_scan64(mine, scratch, &tot);
   for (int e = e0; e < e1; ++e) {
     pre[e] = run;
-    const unsigned long long c = (unsigned)cnt[e];
-    run += c | ((c ? 1ull : 0ull) << 20) |
-           ((c && (int)c < p.dense_min
-                 ? (unsigned long long)(p.I / kTileRows) * ((c + kTileTok - 1) / kTileTok)
-                 : 0ull)
-            << 32);
+    run += packed(e);
   }
   __syncthreads();
+  const int n_local_pairs = (int)(tot & 0xFFFFF);
   const int n_touched = (int)((tot >> 20) & 0xFFF);
   const int routed_items = (int)(tot >> 32);
-  const int n_slots = n_touched + S;
+  const unsigned smask = p.shared_mask;
+  const int n_shared_local = __popc(smask & ((1u << S) - 1u));
+  const int n_slots = n_touched + n_shared_local;
   const int sh_items = B < p.dense_min ? (p.Ish / kTileRows) * ((B + kTileTok - 1) / kTileTok) : 0;
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    if (cnt[e] > 0) {
+    if (cnt[e] > 0 && e >= p.e_begin && e < p.e_end) {
       const unsigned long long pr = pre[e];
       Slot s;
       s.kind = 0;
-      s.expert = e;
+      s.expert = e - p.e_begin;
       s.T = cnt[e];
       s.q0 = (int)(pr & 0xFFFFF);
       s.I = p.I;
@@ -217,20 +220,30 @@ __device__ void group_pairs(const FwdParams& p, uint32_t* dyn, unsigned long lon
       p.slots[(int)((pr >> 20) & 0xFFF)] = s;
     }
   }
+  // local shared expert s_i: slot n_touched + (its rank among the local shared experts)
+  auto shared_slot = [&](int s_i) -> int {
+    return ((smask >> s_i) & 1u) ? n_touched + __popc(smask & ((1u << s_i) - 1u)) : -1;
+  };
   for (int s_i = threadIdx.x; s_i < S; s_i += blockDim.x) {
+    const int j = shared_slot(s_i);
+    if (j < 0) continue;
     Slot s;
     s.kind = 1;
     s.expert = s_i;
     s.T = B;
     s.q0 = B * k + s_i * B;
     s.I = p.Ish;
-    s.item0 = routed_items + s_i * sh_items;
+    s.item0 = routed_items + (j - n_touched) * sh_items;
     s.pad0 = s.pad1 = 0;
-    p.slots[n_touched + s_i] = s;
+    p.slots[j] = s;
   }
   // routed pairs: rank of token t among the tokens of its expert
   for (int pi = threadIdx.x; pi < B * k; pi += blockDim.x) {
     const int t = pi / k, e = sidx[pi];
+    if (e < p.e_begin || e >= p.e_end) {
+      p.pair_index[t * (k + S) + (pi % k)] = -1;
+      continue;
+    }
     int rank = __popc(tokmask[e * W + (t >> 5)] & ((1u << (t & 31)) - 1u));
     for (int w = 0; w < (t >> 5); ++w) rank += __popc(tokmask[e * W + w]);
     const unsigned long long pr = pre[e];
@@ -240,18 +253,21 @@ __device__ void group_pairs(const FwdParams& p, uint32_t* dyn, unsigned long lon
     p.pair_slot[q] = (int)((pr >> 20) & 0xFFF);
     p.pair_index[t * (k + S) + (pi % k)] = q;
   }
+  // the routed pair indices past the local ones belong to no slot
+  for (int q = n_local_pairs + threadIdx.x; q < B * k; q += blockDim.x) p.pair_slot[q] = -1;
   for (int i = threadIdx.x; i < B * S; i += blockDim.x) {
     const int s_i = i / B, t = i % B;
     const int q = B * k + s_i * B + t;
+    const int j = shared_slot(s_i);
     p.pair_token[q] = t;
     p.pair_w[q] = 1.0f;
-    p.pair_slot[q] = n_touched + s_i;
-    p.pair_index[t * (k + S) + k + s_i] = q;
+    p.pair_slot[q] = j;
+    p.pair_index[t * (k + S) + k + s_i] = j < 0 ? -1 : q;
   }
   if (threadIdx.x == 0) {
     p.meta[kMetaSlots] = n_slots;
     p.meta[kMetaPairs] = B * (k + S);
-    p.meta[kMetaGateItems] = routed_items + S * sh_items;
+    p.meta[kMetaGateItems] = routed_items + n_shared_local * sh_items;
     p.meta[kMetaTouched] = n_touched;
   }
 }

@@ -51,6 +51,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
     const int kind = q >= p.B * p.k ? 1 : 0;
     const int I = kind ? p.Ish : p.I;
     const int j = __ldcg(&p.pair_slot[q]);  // the expert's slot, for its union row
+    if (j < 0) continue;  // an expert another handle evaluates (the same for the whole CTA)
     if (threadIdx.x == 0) s_ncand = 0;
     for (int v0 = threadIdx.x;; v0 += 4 * kSelThreads) {
 #pragma unroll
