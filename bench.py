@@ -693,19 +693,22 @@ def run_crossover(args):
             rule = ("topk", s)
             rule_s = rule if shape.n_shared else None
             t = {}
-            for name, dmin in (("sparse", 0), ("dense", 1), ("auto", DEFAULT_DENSE_MIN)):
+            arms = [("sparse", 0), ("dense", 1), ("auto", DEFAULT_DENSE_MIN)]
+            if shape.n_shared:
+                # the shared experts (every token) on the tensor cores, routed experts sparse
+                arms.append(("shared_dense", B))
+            for name, dmin in arms:
                 moe_set_dense_min_tokens(dl.h, dmin)
                 t[name] = statistics.median(
                     timed_calls(dl, xs, rule, rule_s, args.steps, 3, flush, out)) * 1e3
             row = {"workload": shape.name, "batch": B, "sparsity": s,
-                   "tokens_per_expert": round(B * shape.top_k / shape.n_routed, 3),
-                   "sparse_us": round(t["sparse"], 1), "dense_us": round(t["dense"], 1),
-                   "auto_us": round(t["auto"], 1),
-                   "faster": "dense" if t["dense"] < t["sparse"] else "sparse"}
+                   "tokens_per_expert": round(B * shape.top_k / shape.n_routed, 3)}
+            row.update({f"{name}_us": round(v, 1) for name, v in t.items()})
+            row["faster"] = min((v, name) for name, v in t.items() if name != "auto")[1]
             rows.append(row)
             print(json.dumps(row), flush=True)
     dl.close()
-    wins = [r["batch"] for r in rows if r["faster"] == "dense"]
+    wins = [r["batch"] for r in rows if r["faster"] != "sparse"]
     print(json.dumps({"workload": shape.name, "crossover_batch": min(wins) if wins else None,
                       "rows": len(rows)}))
 

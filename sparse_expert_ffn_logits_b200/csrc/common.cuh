@@ -103,7 +103,7 @@ struct FwdParams {
   int* err;            // device error word
   const void* zero_row;  // H zero elements (source of the copies of absent tokens)
   unsigned long long* trace;  // per-CTA phase timestamps (nullptr: tracing off)
-  unsigned* claim;            // [2] work-item counters of the gate and up/down kernels
+  unsigned* claim;            // [3] work-item counters: gate (routed), up/down, gate (shared)
   unsigned* hist;             // [Pmax][kHistBins] score histograms of top-K pairs (zero at rest)
   // roster routing (nullptr: off): the router picks the top-k of logits + router_bias and adds
   // its choice to roster_counts; the weights stay those of the unbiased logits

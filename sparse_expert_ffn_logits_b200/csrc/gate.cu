@@ -87,34 +87,69 @@ __global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, 
   for (int i = threadIdx.x; i < kMetaRing * (int)(sizeof(GateMeta) / 4); i += blockDim.x)
     reinterpret_cast<int*>(s_meta)[i] = 0;  // pointers become null, tokens 0
   pdl_trigger();
-  pdl_wait();
-  trace_point(p.trace, 1, 1);
-  // the slot count and every slot entry that can exist (E + S) in one round trip; entries at
-  // n_slots and beyond are stale and never searched
-  const int n_slots = ld_cg(&p.meta[kMetaSlots]);
-  const int n_items = ld_cg(&p.meta[kMetaGateItems]);
-  load_slot_table(p, min(p.E + p.S, kMaxSlots), s_tab);
   __syncthreads();
   const int H = p.H;
   volatile int* abort = &s_abort;
 
   if (warp == kMetaWarp) {
-    // ---------------- meta: claims items (its own contiguous share first, then a few at a time
-    // from the work counter, so that fast CTAs take more of the tail) and publishes their
-    // records: the row pointer for the copier (mrows), then the tokens for the consumers
-    // (mfull); it also fills the token tiles of the generic variant.  A record with end = 1
-    // closes the stream.
+    // ---------------- meta: claims items and publishes their records: the row pointer for the
+    // copier (mrows), then the tokens for the consumers (mfull); it also fills the token tiles
+    // of the generic variant.  A record with end = 1 closes the stream.
+    // Items come in two spaces.  First the shared experts' items, which need no routing (shared
+    // expert s evaluates every token: token t is pair B k + s B + t), claimed a few at a time
+    // from a counter while the router may still run.  Then, after the wait for the router, the
+    // routed items: a contiguous share of 7/8 of them per CTA (token tiles stay together), the
+    // rest from a second counter in small chunks, so that fast CTAs take more of the tail.
+    // Only this warp reads what the router wrote, so only it waits.
     int xuse[2] = {0, 0};
-    // a contiguous share of 7/8 of the items (token tiles stay together), then the rest from
-    // the counter in small chunks
-    const int share = n_items * 7 / 8 / (int)gridDim.x;
-    const int dyn0 = share * (int)gridDim.x;
-    int cb = blockIdx.x * share, ce = cb + share;
+    const int Bt = (p.B + kTileTok - 1) / kTileTok;
+    const int sh_groups = p.Ish / kTileRows;
+    const bool sh_sparse = p.S > 0 && p.B < p.dense_min;
+    const int n_pre = sh_sparse ? __popc(p.shared_mask) * sh_groups * Bt : 0;
+    int n_slots = 0, n_items = n_pre, share = 0, dyn0 = 0;
+    bool routed_known = false;
+    int cb = 0, ce = 0;
+    auto learn_routing = [&]() {
+      pdl_wait();
+      if (p.trace && lane == 0 && blockIdx.x < kTraceCtas)
+        const_cast<unsigned long long*>(p.trace)[((size_t)1 * kTraceCtas + blockIdx.x) *
+                                                     kTracePoints + 1] = globaltimer();
+      // the slot count and every slot entry that can exist (E + S) in one round trip; entries
+      // at n_slots and beyond are stale and never searched
+      n_slots = ld_cg(&p.meta[kMetaSlots]);
+      const int n_routed = ld_cg(&p.meta[kMetaGateItems]) - n_pre;
+      for (int j = lane; j < min(p.E + p.S, kMaxSlots); j += 32) {
+        const Slot sl = load_slot(&p.slots[j]);
+        s_tab[j] = make_int4(sl.expert | (sl.kind << 16), sl.T, sl.q0, sl.item0);
+      }
+      __syncwarp();
+      share = n_routed * 7 / 8 / (int)gridDim.x;
+      dyn0 = share * (int)gridDim.x;
+      cb = n_pre + blockIdx.x * share;
+      ce = cb + share;
+      n_items = n_pre + n_routed;
+      routed_known = true;
+    };
+    int pre_next = 0, pre_end = 0;
     auto claim = [&]() -> int {
+      if (!routed_known) {
+        if (pre_next >= pre_end) {
+          int b = 0;
+          if (lane == 0 && n_pre > 0) b = (int)atomicAdd(&p.claim[2], (unsigned)kGateChunk);
+          b = __shfl_sync(0xffffffffu, b, 0);
+          if (n_pre > 0 && b < n_pre) {
+            pre_next = b;
+            pre_end = min(b + kGateChunk, n_pre);
+          } else {
+            learn_routing();
+          }
+        }
+        if (!routed_known) return pre_next++;
+      }
       if (cb >= ce) {
         int b = 0;
         if (lane == 0) b = dyn0 + (int)atomicAdd(&p.claim[0], (unsigned)kGateChunk);
-        b = __shfl_sync(0xffffffffu, b, 0);
+        b = __shfl_sync(0xffffffffu, b, 0) + n_pre;
         if (b >= n_items) {
           cb = ce = n_items;
           return -1;
@@ -124,24 +159,45 @@ __global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, 
       }
       return cb++;
     };
-    auto tile_key = [&](int item) -> int {
-      const int j = find_item_slot(s_tab, n_slots, item);
-      const int I = (s_tab[j].x >> 16) ? p.Ish : p.I;
-      return j * 1024 + (item - s_tab[j].w) / (I / kTileRows);
+    // An item's place: slot entry {expert | kind << 16, T, q0, first item} and its local index
+    // within that slot's items.  Shared items carry the local shared expert's entry directly.
+    struct Place {
+      int4 sl;
+      int local, key;
+    };
+    auto place = [&](int item) -> Place {
+      Place pl;
+      if (item < n_pre) {
+        const int o = item / (sh_groups * Bt);  // o-th shared expert of this handle
+        unsigned m = p.shared_mask;
+        for (int i = 0; i < o; ++i) m &= m - 1;
+        const int s_i = __ffs(m) - 1;
+        pl.sl = make_int4(s_i | (1 << 16), p.B, p.B * p.k + s_i * p.B, 0);
+        pl.local = item - o * sh_groups * Bt;
+        pl.key = (1 << 20) + s_i * 1024 + pl.local / sh_groups;
+      } else {
+        const int r = item - n_pre;
+        const int j = find_item_slot(s_tab, n_slots, r);
+        pl.sl = s_tab[j];
+        pl.local = r - pl.sl.w;
+        const int I = (pl.sl.x >> 16) ? p.Ish : p.I;
+        pl.key = j * 1024 + pl.local / (I / kTileRows);
+      }
+      return pl;
     };
     int key = -1, xb = rc.nxb - 1, tok_l = -1, mi = 0;
     int cur = claim();
-    int cur_key = cur >= 0 ? tile_key(cur) : -1;
+    Place cpl = cur >= 0 ? place(cur) : Place{};
     for (; cur >= 0 && !*abort; ++mi) {
       const int nxt = claim();
-      const int nxt_key = nxt >= 0 ? tile_key(nxt) : -1;
+      const Place npl = nxt >= 0 ? place(nxt) : Place{};
+      const int cur_key = cpl.key, nxt_key = nxt >= 0 ? npl.key : -1;
       const int m = mi % kMetaRing;
       if (!mbar_wait(&mempty[m], ((mi / kMetaRing) & 1) ^ 1, abort, p.err)) break;
-      const int j = find_item_slot(s_tab, n_slots, cur);
-      const int4 sl = s_tab[j];
+      const int4 sl = cpl.sl;
       const int kind = sl.x >> 16, ex = sl.x & 0xffff, T = sl.y, q0 = sl.z;
       const int I = kind ? p.Ish : p.I;
-      const int local = cur - sl.w, tt = local / (I / kTileRows), rg = local % (I / kTileRows);
+      const int local = cpl.local, tt = local / (I / kTileRows), rg = local % (I / kTileRows);
       const int nt = min(kTileTok, T - tt * kTileTok);
       if (lane == 0) {  // the copier's part first: it needs no token
         const __nv_bfloat16* base =
@@ -158,7 +214,10 @@ __global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, 
       int xpar = 0;
       if (cur_key != key) {
         key = cur_key;
-        tok_l = lane < nt ? __ldcg(&p.pair_token[q0 + tt * kTileTok + lane]) : -1;
+        // a shared expert's pair q0 + i is token i; a routed pair's token is in the pair table
+        tok_l = lane >= nt ? -1
+                : kind ? tt * kTileTok + lane
+                       : __ldcg(&p.pair_token[q0 + tt * kTileTok + lane]);
         if constexpr (!kReg) {
           xb = (xb + 1) % rc.nxb;
           if (!mbar_wait(&xempty[xb], (xuse[xb] & 1) ^ 1, abort, p.err)) break;
@@ -186,8 +245,9 @@ __global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, 
       __syncwarp();
       if (lane == 0) mbar_arrive(&mfull[m]);
       cur = nxt;
-      cur_key = nxt_key;
+      cpl = npl;
     }
+    if (!routed_known) learn_routing();  // every CTA waits for the router before it exits
     {  // closing record
       const int m = mi % kMetaRing;
       mbar_wait(&mempty[m], ((mi / kMetaRing) & 1) ^ 1, abort, p.err);

@@ -19,7 +19,7 @@ __global__ void finalize_kernel(FwdParams p) {
   trace_point(p.trace, 4, 0);
   pdl_wait();
   trace_point(p.trace, 4, 1);
-  if (blockIdx.x == 0 && threadIdx.x < 2) p.claim[threadIdx.x] = 0;  // work counters, next call
+  if (blockIdx.x == 0 && threadIdx.x < 3) p.claim[threadIdx.x] = 0;  // work counters, next call
   const size_t n4 = (size_t)p.B * p.H / 4;
   float4* acc = reinterpret_cast<float4*>(p.out_acc);
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;

@@ -176,7 +176,7 @@ size_t carve(moe_handle* h, char* base) {
   char* zb = cv.take<char>(0);
   p.tile_ticket = cv.take<unsigned>((Bm + moe::kTileTok - 1) / moe::kTileTok);
   p.global_ticket = cv.take<unsigned>(1);
-  p.claim = cv.take<unsigned>(2);
+  p.claim = cv.take<unsigned>(3);
   p.slot_ticket = cv.take<unsigned>(slots);
   p.ubits = cv.take<uint32_t>(slots * Wm);
   p.hist = cv.take<unsigned>(Pm * moe::kHistBins);

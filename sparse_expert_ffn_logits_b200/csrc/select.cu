@@ -41,9 +41,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
     // The first activations are requested before the pair's slot is known (the row is Imax
     // long whatever the expert's I): one round trip instead of three dependent ones.
     const float4* a4 = reinterpret_cast<const float4*>(p.act + (size_t)q * Imax);
-    float4 f[4];
+    constexpr int kKeyLoads = 8;  // 16-byte loads in flight per thread (I <= 8192 in one round)
+    float4 f[kKeyLoads];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kKeyLoads; ++u) {
       const int v = threadIdx.x + u * kSelThreads;
       f[u] = v < Imax / 4 ? __ldcg(a4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
@@ -53,9 +54,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
     const int j = __ldcg(&p.pair_slot[q]);  // the expert's slot, for its union row
     if (j < 0) continue;  // an expert another handle evaluates (the same for the whole CTA)
     if (threadIdx.x == 0) s_ncand = 0;
-    for (int v0 = threadIdx.x;; v0 += 4 * kSelThreads) {
+    for (int v0 = threadIdx.x;; v0 += kKeyLoads * kSelThreads) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < kKeyLoads; ++u) {
         const int v = v0 + u * kSelThreads;
         if (v < I / 4) {
           const float fv[4] = {f[u].x, f[u].y, f[u].z, f[u].w};
@@ -70,10 +71,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
           }
         }
       }
-      if (v0 + 4 * kSelThreads >= I / 4) break;
+      if (v0 + kKeyLoads * kSelThreads >= I / 4) break;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {  // the next four 16-byte loads per thread
-        const int v = v0 + 4 * kSelThreads + u * kSelThreads;
+      for (int u = 0; u < kKeyLoads; ++u) {  // the next 16-byte loads per thread
+        const int v = v0 + kKeyLoads * kSelThreads + u * kSelThreads;
         f[u] = v < I / 4 ? __ldcg(a4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
@@ -210,13 +211,16 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
       }
     }
     if (q == (int)blockIdx.x) trace_point(p.trace, 2, 3);
-    // Kept set, one ballot per 32-neuron chunk c (neurons 32c .. 32c + 31), written as the
-    // pair's mask row and OR-ed into the expert's union row.  When every key equal to the cut
-    // is kept (the usual case) the mask is simply key >= tau.  Otherwise ties are kept lowest
-    // index first: warp 0 scans the chunks' tie counts in order and trims each chunk's ties.
+    // Kept set, one ballot per 32-neuron chunk c (neurons 32c .. 32c + 31), gathered in shared
+    // memory, then written by all threads at once as the pair's mask row and OR-ed into the
+    // expert's union row.  When every key equal to the cut is kept (the usual case) the mask is
+    // simply key >= tau.  Otherwise ties are kept lowest index first: warp 0 scans the chunks'
+    // tie counts in order and trims each chunk's ties.
     const int nch = I / 32;
     uint32_t* mrow = p.maskbits + (size_t)q * Wmax;
     uint32_t* urow = p.ubits + (size_t)j * Wmax;
+    uint32_t* s_km = key + Imax;        // [Imax / 32] above-cut masks, then the kept masks
+    uint32_t* s_em = s_km + Imax / 32;  // [Imax / 32] tie masks
     if (!radix || eqtot == need) {
       for (int c = warp; c < nch; c += kSelWarps) {
         const uint32_t u = key[32 * c + lane];
@@ -225,14 +229,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
         else if (mode == 1) k_n = __uint_as_float(u) > thr;
         else k_n = K >= I;
         const unsigned km = __ballot_sync(0xffffffffu, k_n);
-        if (lane == 0) {
-          mrow[c] = km;
-          if (km) red_or(&urow[c], km);
-        }
+        if (lane == 0) s_km[c] = km;
       }
     } else {
-      uint32_t* s_km = key + Imax;        // [Imax / 32] above-cut masks, then the kept masks
-      uint32_t* s_em = s_km + Imax / 32;  // [Imax / 32] tie masks
       for (int c = warp; c < nch; c += kSelWarps) {
         const uint32_t u = key[32 * c + lane];
         const unsigned gm = __ballot_sync(0xffffffffu, u > tau);
@@ -264,14 +263,12 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
           tb += ne;
         }
       }
-      __syncthreads();
-      for (int c = warp; c < nch; c += kSelWarps) {
-        if (lane == 0) {
-          const uint32_t km = s_km[c];
-          mrow[c] = km;
-          if (km) red_or(&urow[c], km);
-        }
-      }
+    }
+    __syncthreads();
+    for (int c = threadIdx.x; c < nch; c += kSelThreads) {
+      const uint32_t km = s_km[c];
+      mrow[c] = km;
+      if (km) red_or(&urow[c], km);
     }
     if (q == (int)blockIdx.x) trace_point(p.trace, 2, 4);
     // the last pair of an expert to finish compacts the expert's union (atomic ticket, no
@@ -285,32 +282,37 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
     }
     __syncthreads();
     if (q == (int)blockIdx.x) trace_point(p.trace, 2, 6);
-    if (s_last && warp == 0) {
-      // warp 0 compacts the union bitmask into the ascending row list (lane l takes a
-      // contiguous block of words) and clears it
+    if (s_last) {
+      // The whole CTA compacts the union bitmask into the ascending row list and clears it:
+      // thread t owns the words [t wpt, (t + 1) wpt), a block scan of their bit counts gives
+      // each word's first list position, and then each warp writes one word per step, lane l
+      // placing bit l at its rank among the word's set bits.
       __threadfence();
-      const int W = I / 32, wpl = (W + 31) / 32;
-      const int wb = min(W, lane * wpl), we = min(W, wb + wpl);
+      const int W = I / 32, wpt = (W + kSelThreads - 1) / kSelThreads;
+      uint32_t* s_word = key;               // [W] union words (the keys are no longer needed)
+      int* s_base = reinterpret_cast<int*>(key + Imax / 2);  // [W] first position of each word
+      const int wb = min(W, (int)threadIdx.x * wpt), we = min(W, wb + wpt);
       int c = 0;
-      for (int w = wb; w < we; ++w) c += __popc(__ldcg(&urow[w]));
-      int incl = c;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      int upos = incl - c;
-      int* ul = p.ulist + (size_t)j * Imax;
       for (int w = wb; w < we; ++w) {
-        uint32_t b = __ldcg(&urow[w]);
+        const uint32_t b = __ldcg(&urow[w]);
         urow[w] = 0;
-        while (b) {
-          ul[upos++] = w * 32 + __ffs(b) - 1;
-          b &= b - 1;
-        }
+        s_word[w] = b;
+        c += __popc(b);
       }
-      if (lane == 31) {
-        p.ucnt[j] = incl;
+      int total;
+      int base = block_exclusive_scan(c, reinterpret_cast<int*>(hist), &total);
+      for (int w = wb; w < we; ++w) {
+        s_base[w] = base;
+        base += __popc(s_word[w]);
+      }
+      __syncthreads();
+      int* ul = p.ulist + (size_t)j * Imax;
+      for (int w = warp; w < W; w += kSelWarps) {
+        const uint32_t b = s_word[w];
+        if ((b >> lane) & 1u) ul[s_base[w] + __popc(b & lanemask_lt())] = w * 32 + lane;
+      }
+      if (threadIdx.x == 0) {
+        p.ucnt[j] = total;
         p.slot_ticket[j] = 0;
       }
     }
