@@ -75,6 +75,14 @@ def parse():
     ap.add_argument("--crossover", action="store_true",
                     help="time the sparse kernels against the tensor-core path per batch size "
                          "(one GPU) and print the table instead of the benchmark line")
+    ap.add_argument("--profile", action="store_true",
+                    help="only make warm-up + steps layer calls (L2 flushed before each), for a "
+                         "profiler to capture; prints one summary line")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="routed experts of the layer (default: the workload's); fewer experts "
+                         "keep the same kernels and per-item work with less memory resident")
+    ap.add_argument("--dense-min", type=int, default=DEFAULT_DENSE_MIN,
+                    help="path choice for --profile (see moe_set_dense_min_tokens)")
     return ap.parse_args()
 
 
@@ -193,9 +201,13 @@ def workload_config(shape, B, world, s):
             + (", the same sparsity for the shared experts" if shape.n_shared else "")}
 
 
-def shape_of(name):
+def shape_of(name, experts=None):
     import synth
-    return synth.SHAPES[WORKLOADS.get(name, name)]
+    shape = synth.SHAPES[WORKLOADS.get(name, name)]
+    if experts:
+        shape = shape.with_(name=f"{shape.name}-{experts}e", n_routed=experts,
+                            top_k=min(shape.top_k, experts))
+    return shape
 
 
 def algorithmic_bytes(shape, dbg, B):
@@ -672,6 +684,29 @@ def run_reference(args):
                     "d2h_bytes_per_step": 0}}
 
 
+def run_profile(args):
+    """Warm-up + steps layer calls of one workload (L2 flushed before each) for a profiler."""
+    import torch
+
+    import synth
+    from sparse_expert_ffn_logits_b200 import moe_set_dense_min_tokens
+    from sparse_expert_ffn_logits_b200.workload import DeviceLayer
+    shape = shape_of(args.workload, args.experts)
+    B, rule = args.batch, ("topk", args.sparsity)
+    rule_s = rule if shape.n_shared else None
+    dl = DeviceLayer(shape, max_tokens=B)
+    moe_set_dense_min_tokens(dl.h, args.dense_min)
+    flush = make_flush(torch.device("cuda", 0))
+    xs = [dl.tokens(B, synth.token_seed(shape, i)) for i in range(4)]
+    out = torch.empty_like(xs[0])
+    ms = timed_calls(dl, xs, rule, rule_s, args.steps, args.warmup, flush, out)
+    print(json.dumps({"profile": shape.name, "batch": B, "sparsity": args.sparsity,
+                      "experts": shape.n_routed, "calls": args.warmup + args.steps,
+                      "launches_per_call": dl.last_launches(),
+                      "median_us": round(statistics.median(ms) * 1e3, 1)}))
+    dl.close()
+
+
 def run_crossover(args):
     """Layer time per batch size with the dense tensor-core path off (every expert sparse) and
     forced on (every expert dense), L2 flushed before each call; prints one JSON line per
@@ -724,6 +759,9 @@ def main():
         return 0
     if args.crossover:
         run_crossover(args)
+        return 0
+    if args.profile:
+        run_profile(args)
         return 0
     import torch
     import torch.distributed as dist

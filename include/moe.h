@@ -217,8 +217,11 @@ moe_status moe_debug_force_timeout(moe_handle* h, void* stream);
  * the 0/1 mask and SiLU(g).  bf16 layers only (fp32 layers always take the sparse kernels).
  *   MOE_DENSE_AUTO (-1, the default)  per call: every expert takes the dense path when the
  *                      batch's average tokens per routed expert n_tokens * top_k / n_routed is
- *                      >= 6 (>= 10 when the routed sparsity is above 0.7), else the sparse path;
- *                      thresholds measured on B200
+ *                      >= 6 (>= 10 when the routed sparsity is above 0.7); otherwise, when a
+ *                      shared expert's packed weights exceed the 126 MB L2 cache, the shared
+ *                      experts alone take it from 32 tokens on (128 when the routed sparsity is
+ *                      below 0.3); else every expert takes the sparse path.  Thresholds measured
+ *                      on B200
  *   0                  never the dense path
  *   n > 0              per expert: an expert (routed or shared) with >= n tokens in the call
  *                      takes the dense path, the others the sparse kernels

@@ -426,7 +426,9 @@ __global__ void __launch_bounds__(kThreads) router_cluster_kernel(FwdParams p) {
     if (lane < kTileTok) s_xt[warp][lane] = t0 + lane < B ? x + (size_t)(t0 + lane) * H : nullptr;
     __syncwarp();
     float d[4] = {0.f, 0.f, 0.f, 0.f};
-    tile_dot<4>(wr + (size_t)min(e0 + g, E - 1) * H, wr + (size_t)min(e0 + g + 8, E - 1) * H,
+    // every block of the CTA's slice of H in flight at once (up to 10 x 32 columns: one round
+    // trip to HBM for H <= 5120 with 16 CTAs)
+    tile_dot<10>(wr + (size_t)min(e0 + g, E - 1) * H, wr + (size_t)min(e0 + g + 8, E - 1) * H,
                 s_xt[warp], blo, 1, bhi, d);
 #pragma unroll
     for (int c = 0; c < 4; ++c) {

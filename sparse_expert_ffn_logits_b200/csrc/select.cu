@@ -51,6 +51,16 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
     // routed pairs come first (B * k of them), then the shared experts' pairs
     const int kind = q >= p.B * p.k ? 1 : 0;
     const int I = kind ? p.Ish : p.I;
+    // the pair's score histogram (top-K pairs) is requested together with its activations:
+    // thread r holds the 8 bins counted from the top, [8 (255 - r), 8 (256 - r))
+    const bool hist_on = uses_hist(p, kind);
+    uint4 h0 = make_uint4(0, 0, 0, 0), h1 = make_uint4(0, 0, 0, 0);
+    unsigned* hrow = p.hist + (size_t)q * kHistBins;
+    const int hb0 = 8 * (kSelThreads - 1 - threadIdx.x);
+    if (hist_on) {
+      h0 = __ldcg(reinterpret_cast<const uint4*>(hrow + hb0));
+      h1 = __ldcg(reinterpret_cast<const uint4*>(hrow + hb0 + 4));
+    }
     const int j = __ldcg(&p.pair_slot[q]);  // the expert's slot, for its union row
     if (j < 0) continue;  // an expert another handle evaluates (the same for the whole CTA)
     if (threadIdx.x == 0) s_ncand = 0;
@@ -94,16 +104,13 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
       // most 32 keys share the prefix, one warp ranks them directly.
       uint32_t prefix = 0, pmask = 0;
       int krem = K, cand = I, shift = 28, pass = 0;
-      if (uses_hist(p, kind)) {
-        // The gate counted this pair's keys by their top 12 bits.  Thread r owns the 8 bins
-        // counted from the top, [8 (255 - r), 8 (256 - r)); an exclusive scan in thread order
-        // gives the keys in the bins above them, and the thread whose bins hold the K-th largest
-        // key names its bin.  The row is cleared for the next call.
+      if (hist_on) {
+        // The gate counted this pair's keys by their top 12 bits.  An exclusive scan of the
+        // threads' bin sums in thread order gives the keys in the bins above each thread's
+        // bins, and the thread whose bins hold the K-th largest key names its bin.  The row is
+        // cleared for the next call.
         static_assert(kHistBins == 8 * kSelThreads, "8 histogram bins per thread");
-        unsigned* hrow = p.hist + (size_t)q * kHistBins;
-        const int b0 = 8 * (kSelThreads - 1 - threadIdx.x);
-        const uint4 h0 = __ldcg(reinterpret_cast<const uint4*>(hrow + b0));
-        const uint4 h1 = __ldcg(reinterpret_cast<const uint4*>(hrow + b0 + 4));
+        const int b0 = hb0;
         *reinterpret_cast<uint4*>(hrow + b0) = make_uint4(0, 0, 0, 0);
         *reinterpret_cast<uint4*>(hrow + b0 + 4) = make_uint4(0, 0, 0, 0);
         const unsigned hb[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};

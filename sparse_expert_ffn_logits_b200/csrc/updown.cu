@@ -102,6 +102,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
   __shared__ int s_abort;
   __shared__ UdMeta s_meta[kMetaRing];
   __shared__ __align__(16) uint32_t s_hcw[2][kTileTok][kTileRows / 2];
+  __shared__ uint32_t s_tmem;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + rc.ns;
   uint64_t* mfull = empty + rc.ns;
@@ -135,6 +136,18 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
   }
   for (int i = threadIdx.x; i < kMetaRing * (int)(sizeof(UdMeta) / 4); i += blockDim.x)
     reinterpret_cast<int*>(s_meta)[i] = 0;
+  // Down-projection accumulators in tensor memory: consumer warp w keeps the 16 values of each
+  // of its 64-column sub-chunks (spw per stage, nk stages) in lane quarter w % 4, columns
+  // 256 (w / 4) + 16 (kc spw + local sub-chunk), while consecutive items of one (expert, token
+  // tile) follow each other, and flushes them to the output accumulator once per such run.
+  // Hidden sizes that would need more than 256 columns per warp group reduce every item.
+  const int spw = (rc.kc / 64 + kWarps - 1) / kWarps;
+  const bool tmem_acc = rc.nk * spw * 16 <= 256;
+  if (tmem_acc && warp == 0) tmem_alloc(&s_tmem, 512);
+  tmem_fence_before();
+  __syncthreads();
+  tmem_fence_after();
+  const uint32_t tmem_base = tmem_acc ? s_tmem : 0u;
   pdl_trigger();
   pdl_wait();
   trace_point(p.trace, 3, 1);
@@ -367,8 +380,9 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
   // ---------------- consumers
   constexpr int kXR = kReg ? NK : 1, kXB = kReg ? BPW : 1;
   uint4 xr[kXR][kXB];
-  int it = 0, ib = 0, cur = -1;
+  int it = 0, ib = 0, cur = -1, run_key = -1;
   const int nblk = rc.kc / 32, nsub = rc.kc / 64;
+  const uint32_t tmem_warp = tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + 256u * (warp >> 2);
   const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(p.x);
   for (int mi = 0;; ++mi) {
     const int m = mi % kMetaRing;
@@ -385,6 +399,8 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
     const UdMeta& mt = s_meta[m];
     const int xb = min(max(mt.xb, 0), max(rc.nxb - 1, 0));  // a record is trusted only w/o abort
     const int xlast = mt.xlast;
+    const int item_key = mt.key;  // the record is handed back to the meta warp before the down
+                                  // projection: everything read from it is read here
     const int tok0 = mt.tok[2 * t], tok1 = mt.tok[2 * t + 1];
     const float w0 = mt.w[2 * t], w1 = mt.w[2 * t + 1];
     const unsigned char* xrow = xbuf + xb * rc.xs_bytes + g * rc.xs_stride;
@@ -463,8 +479,11 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
     }
     consumer_sync(kThreads);
     if (lane == 0) mbar_arrive(&mempty[m]);
-    // 3-4. down projection of each stage's 64-column sub-chunks, reduced into out_acc
+    // 3-4. down projection of each stage's 64-column sub-chunks, kept in tensor memory while
+    // the run of items of this (expert, token tile) goes on, reduced into out_acc at its end
     const uint32_t b0 = s_hcw[ib][g][t], b1 = s_hcw[ib][g][4 + t];
+    const bool first = item_key != run_key, last = xlast != 0 || !tmem_acc;
+    run_key = last ? -1 : item_key;
     for (int kc = 0; kc < rc.nk; ++kc, ++it) {
       const int st = it % rc.ns;
       mbar_wait(&full[st], (it / rc.ns) & 1, abort, p.err);
@@ -488,12 +507,30 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
                     __byte_perm(w0v[i], w1v[i], 0x7632), __byte_perm(w2v[i], w3v[i], 0x5410),
                     __byte_perm(w2v[i], w3v[i], 0x7632), b0, b1);
         }
-        if (!aborted && tok0 >= 0) {
+        if (!(first && last)) {
+          float v[16];
+          const uint32_t col = tmem_warp + 16u * (uint32_t)(kc * spw + (sc - warp) / kWarps);
+          if (!first) {  // earlier items of the run, summed in the same order every time
+            tmem_ld16(col, v);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+              for (int c = 0; c < 4; ++c) acc[i][c] += v[4 * i + c];
+          }
+          if (!last) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+              for (int c = 0; c < 4; ++c) v[4 * i + c] = acc[i][c];
+            tmem_st16(col, v);
+          }
+        }
+        if (last && !aborted && tok0 >= 0) {
           float* o = p.out_acc + (size_t)tok0 * H + hb;
           red_add_v4(o, w0 * acc[0][0], w0 * acc[0][2], w0 * acc[1][0], w0 * acc[1][2]);
           red_add_v4(o + 4, w0 * acc[2][0], w0 * acc[2][2], w0 * acc[3][0], w0 * acc[3][2]);
         }
-        if (!aborted && tok1 >= 0) {
+        if (last && !aborted && tok1 >= 0) {
           float* o = p.out_acc + (size_t)tok1 * H + hb;
           red_add_v4(o, w1 * acc[0][1], w1 * acc[0][3], w1 * acc[1][1], w1 * acc[1][3]);
           red_add_v4(o + 4, w1 * acc[2][1], w1 * acc[2][3], w1 * acc[3][1], w1 * acc[3][3]);
@@ -502,10 +539,16 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);
     }
+    if (!last) tmem_wait_st();  // the next item of the run loads these columns
     if (mi == 0) trace_point(p.trace, 3, 4);
     ib ^= 1;
   }
   trace_point(p.trace, 3, 7);
+  // every consumer warp is done with tensor memory before warp 0 frees it
+  tmem_fence_before();
+  consumer_sync(kThreads);
+  tmem_fence_after();
+  if (tmem_acc && warp == 0) tmem_dealloc(tmem_base, 512);
 }
 
 // fp32 variant: register loads, same items and fragment layout.

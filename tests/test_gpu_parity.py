@@ -9,7 +9,7 @@ import oracle
 import synth
 from sparse_expert_ffn_logits_b200 import (MOE_ERR_DEVICE, MOE_ERR_TIMEOUT, MOE_OK,
                                            moe_debug_force_timeout, moe_get_error,
-                                           moe_set_dense_min_tokens)
+                                           moe_last_launches, moe_set_dense_min_tokens)
 from sparse_expert_ffn_logits_b200.workload import DeviceLayer
 from tests import parity
 
@@ -238,12 +238,19 @@ def llama4_shared():
 
 
 def test_llama4_large_batch(llama4, llama4_shared):
-    # routing and kept sets of every token; the output of sampled tokens
+    # routing and kept sets of every token; the output of sampled tokens.  At these sizes the
+    # automatic path choice puts the shared expert (every token) on the tensor cores and keeps
+    # the routed experts sparse.
     cache = {}
     _run(llama4, 256, ("topk", 0.9), ("topk", 0.9), batch_index=99, tokens=[0, 77, 255],
          shared_weights=llama4_shared, expert_cache=cache)
+    assert moe_last_launches(llama4.h) == 9
+    # Allowance: two of the 128 pairs, both of the shared expert (tokens 27 and 28, neurons
+    # 5689 and 7868), swap a neuron across the cut: oracle gaps 3.0e-6 and 1.6e-6 against a band
+    # of 1e-6 * |cut| (cut ~0.27), inside the fp32 bound of the 5120-term tensor-core gate
+    # (3.1e-2 and 3.05e-2).
     _run(llama4, 64, ("topk", 0.5), ("topk", 0.5), batch_index=98, tokens=[1, 33, 63],
-         shared_weights=llama4_shared, expert_cache=cache)
+         shared_weights=llama4_shared, expert_cache=cache, allow_fp32_bound=2)
 
 
 @pytest.mark.parametrize("B,s", [(64, 0.9), (256, 0.5)])
