@@ -371,8 +371,13 @@ def sweep_rows(dl, batches, rules, peak, flush, pool_n, token_stream_of, steps=2
             rows.append(row)
             times[(kind, s, s_sh)] = (ms, row)
         for (kind, s, s_sh), (ms, row) in times.items():
-            if kind == "topk" and s == 0.9 and ("topk", 0.0, s_sh) in times:
-                row["speedup_s0.9_vs_s0"] = round(times[("topk", 0.0, s_sh)][0] / ms, 3)
+            if kind != "topk" or s != 0.9:
+                continue
+            # against sparsity 0 with the same shared sparsity (DeepSeek-V2-Lite's grid), or with
+            # the shared experts dense too where the grid moves both together (Llama-4's)
+            base = ("topk", 0.0, s_sh) if ("topk", 0.0, s_sh) in times else ("topk", 0.0, 0.0)
+            if base in times:
+                row["speedup_s0.9_vs_s0"] = round(times[base][0] / ms, 3)
         del bx, out
     return rows
 
@@ -700,10 +705,18 @@ def run_profile(args):
     xs = [dl.tokens(B, synth.token_seed(shape, i)) for i in range(4)]
     out = torch.empty_like(xs[0])
     ms = timed_calls(dl, xs, rule, rule_s, args.steps, args.warmup, flush, out)
+    launches = dl.last_launches()
+    # the algorithmic bytes of each token batch (call i used batch i % 4), per stage
+    per_batch = []
+    for x in xs:
+        dl.forward(x, rule, rule_s, out=out)
+        ab = algorithmic_bytes(shape, dl.debug(B), B)
+        per_batch.append({k: int(v) for k, v in ab.items()})
     print(json.dumps({"profile": shape.name, "batch": B, "sparsity": args.sparsity,
                       "experts": shape.n_routed, "calls": args.warmup + args.steps,
-                      "launches_per_call": dl.last_launches(),
-                      "median_us": round(statistics.median(ms) * 1e3, 1)}))
+                      "launches_per_call": launches,
+                      "median_us": round(statistics.median(ms) * 1e3, 1),
+                      "algorithmic_bytes_by_batch": per_batch}))
     dl.close()
 
 

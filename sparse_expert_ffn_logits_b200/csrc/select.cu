@@ -19,10 +19,14 @@
 namespace moe {
 namespace {
 
-constexpr int kSelThreads = 256;
-constexpr int kSelWarps = kSelThreads / 32;
-
-__global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
+// NT threads per pair: 256, or 1024 for intermediate sizes of 4096 and more.  The kernel is
+// latency-bound (dependent shared-memory and warp-level steps), so a large pair gets more warps
+// to hide the latencies and fewer keys per thread in each pass.
+template <int NT>
+__global__ void __launch_bounds__(NT) select_kernel(FwdParams p) {
+  constexpr int kSelThreads = NT, kSelWarps = NT / 32;
+  constexpr int kBpt = kHistBins / NT;  // histogram bins per thread (8 or 2)
+  static_assert(kBpt == 8 || kBpt == 2, "histogram bins per thread");
   extern __shared__ uint32_t sm[];
   __shared__ int hist[2 * kSelWarps * 8];
   __shared__ uint32_t cbuf[32];
@@ -52,14 +56,23 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
     const int kind = q >= p.B * p.k ? 1 : 0;
     const int I = kind ? p.Ish : p.I;
     // the pair's score histogram (top-K pairs) is requested together with its activations:
-    // thread r holds the 8 bins counted from the top, [8 (255 - r), 8 (256 - r))
+    // thread r holds the kBpt bins counted from the top, [kBpt (NT - 1 - r), kBpt (NT - r))
     const bool hist_on = uses_hist(p, kind);
-    uint4 h0 = make_uint4(0, 0, 0, 0), h1 = make_uint4(0, 0, 0, 0);
+    unsigned hb[kBpt];
     unsigned* hrow = p.hist + (size_t)q * kHistBins;
-    const int hb0 = 8 * (kSelThreads - 1 - threadIdx.x);
-    if (hist_on) {
-      h0 = __ldcg(reinterpret_cast<const uint4*>(hrow + hb0));
-      h1 = __ldcg(reinterpret_cast<const uint4*>(hrow + hb0 + 4));
+    const int hb0 = kBpt * (kSelThreads - 1 - threadIdx.x);
+    if constexpr (kBpt == 8) {
+      uint4 h0 = make_uint4(0, 0, 0, 0), h1 = make_uint4(0, 0, 0, 0);
+      if (hist_on) {
+        h0 = __ldcg(reinterpret_cast<const uint4*>(hrow + hb0));
+        h1 = __ldcg(reinterpret_cast<const uint4*>(hrow + hb0 + 4));
+      }
+      hb[0] = h0.x; hb[1] = h0.y; hb[2] = h0.z; hb[3] = h0.w;
+      hb[4] = h1.x; hb[5] = h1.y; hb[6] = h1.z; hb[7] = h1.w;
+    } else {
+      uint2 h0 = make_uint2(0, 0);
+      if (hist_on) h0 = __ldcg(reinterpret_cast<const uint2*>(hrow + hb0));
+      hb[0] = h0.x; hb[1] = h0.y;
     }
     const int j = __ldcg(&p.pair_slot[q]);  // the expert's slot, for its union row
     if (j < 0) continue;  // an expert another handle evaluates (the same for the whole CTA)
@@ -109,18 +122,16 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
         // threads' bin sums in thread order gives the keys in the bins above each thread's
         // bins, and the thread whose bins hold the K-th largest key names its bin.  The row is
         // cleared for the next call.
-        static_assert(kHistBins == 8 * kSelThreads, "8 histogram bins per thread");
         const int b0 = hb0;
-        *reinterpret_cast<uint4*>(hrow + b0) = make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4*>(hrow + b0 + 4) = make_uint4(0, 0, 0, 0);
-        const unsigned hb[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+#pragma unroll
+        for (int i = 0; i < kBpt; ++i) hrow[b0 + i] = 0;
         int mine = 0;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mine += (int)hb[i];
+        for (int i = 0; i < kBpt; ++i) mine += (int)hb[i];
         int above = block_exclusive_scan(mine, reinterpret_cast<int*>(hist), nullptr);
         if (above < K && above + mine >= K) {
 #pragma unroll
-          for (int i = 7; i >= 0; --i) {
+          for (int i = kBpt - 1; i >= 0; --i) {
             const int c = (int)hb[i];
             if (above < K && above + c >= K) {
               s_tau = (uint32_t)(b0 + i);
@@ -334,18 +345,29 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(FwdParams p) {
 // keys [Imax] | kept masks, tie masks [Imax / 32] each
 size_t select_smem_bytes(int imax) { return (size_t)imax * 4 + (size_t)(imax / 32) * 8 + 16; }
 
+// 1024 threads per pair from this intermediate size on
+constexpr int kWideSelect = 4096;
+
 cudaError_t launch_select(const FwdParams& p, const LaunchShape& ls, cudaStream_t st, bool pdl) {
   const int pairs = p.B * (p.k + p.S);
   const int grid = pairs < ls.grid_select ? pairs : ls.grid_select;
-  return launch_pdl(select_kernel, dim3(grid), dim3(kSelThreads), select_smem_bytes(p.Imax), st,
+  if (p.Imax >= kWideSelect)
+    return launch_pdl(select_kernel<1024>, dim3(grid), dim3(1024), select_smem_bytes(p.Imax), st,
+                      pdl, p);
+  return launch_pdl(select_kernel<256>, dim3(grid), dim3(256), select_smem_bytes(p.Imax), st,
                     pdl, p);
 }
 
 cudaError_t configure_select(int imax, int budget, int* occupancy) {
   const size_t smem = select_smem_bytes(imax);
-  cudaError_t e = allow_max_smem(select_kernel, budget);
+  cudaError_t e = allow_max_smem(select_kernel<256>, budget);
+  if (e == cudaSuccess) e = allow_max_smem(select_kernel<1024>, budget);
   if (e != cudaSuccess) return e;
-  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occupancy, select_kernel, kSelThreads, smem);
+  return imax >= kWideSelect
+             ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(occupancy, select_kernel<1024>, 1024,
+                                                             smem)
+             : cudaOccupancyMaxActiveBlocksPerMultiprocessor(occupancy, select_kernel<256>, 256,
+                                                             smem);
 }
 
 }  // namespace moe
