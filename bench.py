@@ -83,6 +83,9 @@ def parse():
                          "keep the same kernels and per-item work with less memory resident")
     ap.add_argument("--dense-min", type=int, default=DEFAULT_DENSE_MIN,
                     help="path choice for --profile (see moe_set_dense_min_tokens)")
+    ap.add_argument("--no-fused", dest="fused", action="store_false", default=True,
+                    help="run the chain of separate kernels instead of the fused layer kernel "
+                         "(see moe_set_fused)")
     return ap.parse_args()
 
 
@@ -401,6 +404,7 @@ def run_cuda(args, rank, world, local_rank):
     rule = ("topk", s)
     rule_s = rule if shape.n_shared else None
     dl = DeviceLayer(shape, max_tokens=max_tokens, device=dev)
+    dl.set_fused(args.fused)
     pool_n = 32
 
     def pool(nb):
@@ -440,21 +444,32 @@ def run_cuda(args, rank, world, local_rank):
     total_ms = job_time_ms(sum(step_ms), world, dev)
     value = job_throughput(world, B, args.steps, total_ms)
 
-    # ---- per-stage durations (kernels launched back to back, events between them)
-    stage_evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)]
-    for e in stage_evs:
-        e.record()
-    torch.cuda.synchronize()
-    moe_profile_stages(dl.h, stage_evs)
-    stage_ms = {n: [] for n in STAGES}
+    # ---- per-stage durations (kernels launched back to back, events between them).  A call on
+    # the fused layer kernel (3 launches) has router, layer and output cast: the layer's events
+    # are the gate stage's.  The chain of separate kernels is timed too, for its breakdown.
+    fused_call = launches == 3
     nprof = min(args.steps, 20)
-    for i in range(nprof):
-        flush()
-        dl.forward(xs[i % pool_n], rule, rule_s, out=out)
+
+    def stage_times(fused):
+        dl.set_fused(fused)
+        stage_evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)]
+        for e in stage_evs:
+            e.record()
         torch.cuda.synchronize()
-        for j, n in enumerate(STAGES):
-            stage_ms[n].append(stage_evs[j].elapsed_time(stage_evs[j + 1]))
-    moe_profile_stages(dl.h, None)
+        moe_profile_stages(dl.h, stage_evs)
+        stage_ms = {n: [] for n in STAGES}
+        for i in range(nprof):
+            flush()
+            dl.forward(xs[i % pool_n], rule, rule_s, out=out)
+            torch.cuda.synchronize()
+            for j, n in enumerate(STAGES):
+                stage_ms[n].append(stage_evs[j].elapsed_time(stage_evs[j + 1]))
+        moe_profile_stages(dl.h, None)
+        dl.set_fused(args.fused)
+        return {n: statistics.mean(v) for n, v in stage_ms.items()}
+
+    stage_avg = stage_times(args.fused)
+    chain_avg = stage_times(False) if fused_call else stage_avg
     abytes = {n: 0.0 for n in STAGES}
     nb = min(pool_n, nprof, 8)
     for i in range(nb):
@@ -462,20 +477,29 @@ def run_cuda(args, rank, world, local_rank):
         ab = algorithmic_bytes(shape, dl.debug(B), B)
         for n in STAGES:
             abytes[n] += ab[n] / nb
-    stage_avg = {n: statistics.mean(v) for n, v in stage_ms.items()}
-    dom = max(STAGES, key=lambda n: stage_avg[n])
+    if fused_call:  # gate, selection and up/down are one kernel
+        dom = "layer"
+        dom_ms = stage_avg["gate"]
+        dom_bytes = abytes["gate"] + abytes["updown"]
+    else:
+        dom = max(STAGES, key=lambda n: stage_avg[n])
+        dom_ms = stage_avg[dom]
+        dom_bytes = abytes[dom]
     peak, peak_kind = peaks()
-    achieved = abytes[dom] / (stage_avg[dom] / 1e3) / 1e9
+    achieved = dom_bytes / (dom_ms / 1e3) / 1e9
     layer_bytes = sum(abytes[n] for n in ("router", "gate", "updown"))
     traffic = traffic_of(f"{shape.name}:B{B}:s{s}:{dom}")
     layer_gbs = layer_bytes / (total_ms / args.steps / 1e3) / 1e9
+    stage_names = (("router", "router"), ("gate", "layer"), ("finalize", "finalize")) \
+        if fused_call else tuple((n, n) for n in STAGES)
     roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
                 "peak_source": f"hbm copy, {peak_kind}", "unit": "GB/s",
                 "frac": round(achieved / peak, 4),
                 "frac_spec": round(achieved / HBM_SPEC_GBS, 4), "traffic": traffic,
-                "algorithmic_bytes_per_launch": int(abytes[dom]),
-                "launch_us": round(stage_avg[dom] * 1e3, 2),
-                "stages_us": {n: round(v * 1e3, 2) for n, v in stage_avg.items()},
+                "algorithmic_bytes_per_launch": int(dom_bytes),
+                "launch_us": round(dom_ms * 1e3, 2),
+                "stages_us": {out_n: round(stage_avg[n] * 1e3, 2) for n, out_n in stage_names},
+                "chain_stages_us": {n: round(v * 1e3, 2) for n, v in chain_avg.items()},
                 "layer": {"algorithmic_bytes": int(layer_bytes), "gbs": round(layer_gbs, 1),
                           "frac": round(layer_gbs / peak, 4),
                           "frac_spec": round(layer_gbs / HBM_SPEC_GBS, 4)}}
@@ -540,6 +564,7 @@ def run_cuda(args, rank, world, local_rank):
                 sdl = dl
             else:
                 sdl = DeviceLayer(synth.SHAPES[name], max_tokens=max(bs), device=dev)
+                sdl.set_fused(args.fused)
             try:
                 sweep += sweep_rows(sdl, bs, rules, peak, flush, pool_n,
                                     lambda i: token_stream(rank, i))
@@ -701,6 +726,7 @@ def run_profile(args):
     rule_s = rule if shape.n_shared else None
     dl = DeviceLayer(shape, max_tokens=B)
     moe_set_dense_min_tokens(dl.h, args.dense_min)
+    dl.set_fused(args.fused)
     flush = make_flush(torch.device("cuda", 0))
     xs = [dl.tokens(B, synth.token_seed(shape, i)) for i in range(4)]
     out = torch.empty_like(xs[0])

@@ -186,7 +186,9 @@ moe_status moe_debug_lists(moe_handle* h, int n_tokens, int* idx, float* w, floa
  * timing off.  While set, every moe_forward records events[0] before its first kernel and
  * events[i] after its i-th kernel (1 router+top-k+grouping, 2 gate, 3 select, 4 up/down,
  * 5 output cast), and launches the kernels without programmatic overlap so that the interval
- * between consecutive events is that kernel alone.  The handle keeps the event handles, not
+ * between consecutive events is that kernel alone.  A call on the fused layer kernel
+ * (moe_set_fused) records events 2, 3 and 4 after it: its duration is the gate stage's, the
+ * selection and up/down stages are empty.  The handle keeps the event handles, not
  * copies; the caller owns and destroys them. */
 #define MOE_STAGE_EVENTS 6
 moe_status moe_profile_stages(moe_handle* h, void* const* events, int n_events);
@@ -228,6 +230,19 @@ moe_status moe_debug_force_timeout(moe_handle* h, void* stream);
  * INVALID_ARG for a NULL handle or a value below -1.  Takes effect from the next moe_forward. */
 #define MOE_DENSE_AUTO (-1)
 moe_status moe_set_dense_min_tokens(moe_handle* h, int min_tokens);
+
+/* Fused layer kernel ("Uncovering Intra-expert Activation Sparsity ...", technical summary, Key
+ * contributions: the layer stays one fused, graph-capturable unit).  enable = 1 (the default):
+ * a bf16 call whose slots all take the sparse kernels, on a hidden size with register token
+ * fragments (512, 2048, 2880, 5120), runs gate, selection and up/down as one persistent kernel
+ * between the router and the output cast (3 launches instead of 5): a token tile's selections
+ * start as soon as its gate rows are done and an expert's up/down as soon as its union is known.
+ * enable = 0: always the chain of separate kernels.  The results are the same within rounding of
+ * the fp32 output sums (the up/down runs accumulate in another grouping); routing and kept sets
+ * are identical.  Under stage timing (moe_profile_stages) the fused kernel's duration is the
+ * gate stage's, and the selection and up/down stages are empty.  INVALID_ARG for a
+ * NULL handle or enable outside {0, 1}.  Takes effect from the next moe_forward. */
+moe_status moe_set_fused(moe_handle* h, int enable);
 
 /* Expert parallelism ("Uncovering Intra-expert Activation Sparsity ...", technical summary,
  * Methodology: the serving system keeps expert parallelism).  Each of G ranks holds a handle of

@@ -57,7 +57,7 @@ _LIB = None
 EXPORTS = ("moe_create", "moe_packed_bytes", "moe_pack_experts", "moe_forward",
            "moe_forward_roster",
            "moe_forward_host", "moe_debug_lists", "moe_profile_stages", "moe_read_trace",
-           "moe_get_error", "moe_debug_force_timeout", "moe_set_dense_min_tokens",
+           "moe_get_error", "moe_debug_force_timeout", "moe_set_dense_min_tokens", "moe_set_fused",
            "moe_last_launches", "moe_set_expert_range", "moe_forward_partial",
            "moe_cast_output", "moe_destroy",
            "moe_route_noalloc",
@@ -94,6 +94,7 @@ def _lib():
         lib.moe_get_error.argtypes = [P, ctypes.POINTER(I)]
         lib.moe_destroy.argtypes = [P]
         lib.moe_set_dense_min_tokens.argtypes = [P, I]
+        lib.moe_set_fused.argtypes = [P, I]
         lib.moe_last_launches.argtypes = [P, ctypes.POINTER(I)]
         lib.moe_set_expert_range.argtypes = [P, I, I, ctypes.c_uint]
         lib.moe_forward_partial.argtypes = fwd
@@ -256,6 +257,12 @@ def moe_set_dense_min_tokens(h, min_tokens):
     token threshold (see include/moe.h)."""
     _check(_lib().moe_set_dense_min_tokens(ctypes.c_void_p(h) if h else None, int(min_tokens)),
            "moe_set_dense_min_tokens")
+
+
+def moe_set_fused(h, enable):
+    """1: gate, selection and up/down as one fused kernel where it applies (the default); 0: the
+    chain of separate kernels (see include/moe.h)."""
+    _check(_lib().moe_set_fused(ctypes.c_void_p(h) if h else None, int(enable)), "moe_set_fused")
 
 
 def moe_last_launches(h):

@@ -10,7 +10,7 @@ ROOT = os.path.dirname(HERE)
 INCLUDE = os.path.join(ROOT, "include")
 SO = os.path.join(HERE, "libsparse_moe.so")
 OBJ = os.path.join(ROOT, "_build", "sparse_moe")
-SOURCES = ["moe_api.cu", "router.cu", "gate.cu", "select.cu", "updown.cu", "misc.cu",
+SOURCES = ["moe_api.cu", "router.cu", "gate.cu", "select.cu", "updown.cu", "layer.cu", "misc.cu",
            "route_noalloc.cu", "dense.cu"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
               "-Xcompiler", "-fPIC", "-I", INCLUDE, "-Xptxas", "-warn-spills"]

@@ -114,6 +114,12 @@ struct FwdParams {
   int imax_pad;               // Imax rounded up to 128 (row length of hbuf)
   __nv_bfloat16* xp;          // [Pmax][H] x rows of the pairs of dense slots
   __nv_bfloat16* hbuf;        // [Pmax][imax_pad] mask * SiLU(g) * u of dense slots, bf16
+  // fused layer kernel: readiness of the work that depends on other CTAs (zero at rest)
+  unsigned* tile_done;        // [Pmax] gate items finished per token tile, at its first pair
+  int* s_task;                // [Pmax] selection tasks in the order they became ready: pair + 1
+  unsigned* fq;               // [4] selection tasks reserved, claimed; up/down items claimed
+  unsigned long long* u_res;  // [1] up/down entries published << 32 | up/down items reserved
+  int4* u_ent;                // [E+S] per entry: {slot + 1, first item, items, union rows}
 };
 
 // Phase timestamps for tracing: kernel k, CTA b, point i (i < kTracePoints).

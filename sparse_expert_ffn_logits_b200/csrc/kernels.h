@@ -17,6 +17,7 @@ struct LaunchShape {
   int grid_select;    // cap of the selection grid
   Ring ring_gate;     // copy ring of the bf16 gate kernel
   Ring ring_ud;       // copy ring of the bf16 up/down kernel
+  Ring ring_layer;    // copy ring of the fused layer kernel (ns = 0: not available)
   int variant;        // register-fragment ring variant (0: generic token tiles in smem)
   int router_cluster; // CTAs of the single-cluster router (0: only the multi-CTA router)
 };
@@ -44,12 +45,16 @@ cudaError_t launch_updown(const FwdParams& p, int dtype, const LaunchShape& ls, 
 cudaError_t launch_dense(const FwdParams& p, const LaunchShape& ls, int stage, cudaStream_t st,
                          bool pdl);
 cudaError_t configure_dense(int budget);
+// fused layer kernel (layer.cu): gate, selection and up/down in one persistent launch
+bool layer_available(const LaunchShape& ls);
+cudaError_t launch_layer(const FwdParams& p, const LaunchShape& ls, cudaStream_t st, bool pdl);
+cudaError_t configure_layer(int H, int imax, int n_slot_max, int smem_budget, LaunchShape* ls);
 cudaError_t launch_finalize(const FwdParams& p, int dtype, const LaunchShape& ls, cudaStream_t st,
                             bool pdl);
 
 // Set-up (called once per handle, under setup_mutex): shared-memory limits and persistent grid
 // sizes.
-cudaError_t configure_kernels(int dtype, int imax, int max_E, int max_B, int H, LaunchShape* ls);
+cudaError_t configure_kernels(int dtype, int imax, int n_slot_max, int max_B, int H, LaunchShape* ls);
 cudaError_t configure_router(int budget, int* cluster_out);
 size_t router_smem_bytes(int E, int B);
 size_t select_smem_bytes(int imax);

@@ -20,6 +20,16 @@ __global__ void finalize_kernel(FwdParams p) {
   pdl_wait();
   trace_point(p.trace, 4, 1);
   if (blockIdx.x == 0 && threadIdx.x < 3) p.claim[threadIdx.x] = 0;  // work counters, next call
+  // the fused layer kernel's readiness state, for the next call
+  const int n_pairs = p.B * (p.k + p.S);
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_pairs; i += gridDim.x * blockDim.x) {
+    p.tile_done[i] = 0;
+    p.s_task[i] = 0;
+  }
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.E + p.S; i += gridDim.x * blockDim.x)
+    p.u_ent[i] = make_int4(0, 0, 0, 0);
+  if (blockIdx.x == 0 && threadIdx.x < 4) p.fq[threadIdx.x] = 0;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *p.u_res = 0ull;
   const size_t n4 = (size_t)p.B * p.H / 4;
   float4* acc = reinterpret_cast<float4*>(p.out_acc);
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
@@ -262,7 +272,7 @@ unsigned long long current_context_id() {
   return id;
 }
 
-cudaError_t configure_kernels(int dtype, int imax, int max_E, int max_B, int H, LaunchShape* ls) {
+cudaError_t configure_kernels(int dtype, int imax, int n_slot_max, int max_B, int H, LaunchShape* ls) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -284,6 +294,10 @@ cudaError_t configure_kernels(int dtype, int imax, int max_E, int max_B, int H, 
   if (dtype == 0) {
     e = configure_dense(budget);
     if (e != cudaSuccess) return e;
+    e = configure_layer(H, imax, n_slot_max, budget, ls);
+    if (e != cudaSuccess) return e;
+  } else {
+    ls->ring_layer.ns = 0;
   }
   return cudaGetLastError();
 }

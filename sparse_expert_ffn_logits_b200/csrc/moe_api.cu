@@ -48,6 +48,7 @@ struct moe_handle {
   float* roster_bias;  // device [max_tokens][E]: the roster bias of the current call
   int e_begin, e_end;     // routed experts this handle evaluates (all by default)
   unsigned shared_mask;   // shared experts this handle evaluates (all by default)
+  bool fused;             // the fused layer kernel where it applies (default on)
 };
 
 namespace {
@@ -198,6 +199,11 @@ size_t carve(moe_handle* h, char* base) {
   p.slot_ticket = cv.take<unsigned>(slots);
   p.ubits = cv.take<uint32_t>(slots * Wm);
   p.hist = cv.take<unsigned>(Pm * moe::kHistBins);
+  p.tile_done = cv.take<unsigned>(Pm);
+  p.s_task = cv.take<int>(Pm);
+  p.fq = cv.take<unsigned>(4);
+  p.u_res = cv.take<unsigned long long>(1);
+  p.u_ent = cv.take<int4>(slots);
   p.out_acc = cv.take<float>(Bm * c.hidden);
   h->zero_begin = zb;
   h->zero_bytes = (size_t)((base + cv.off) - zb);
@@ -275,16 +281,25 @@ moe_status forward_impl(moe_handle* h, const void* x, int n_tokens, const void* 
       e = moe::launch_roster_bias(roster->counts, roster->pinned, n_tokens, c.n_routed, roster->m,
                                   roster->delta, h->roster_bias, st);
   }
+  // The fused layer kernel does gate, selection and up/down in one launch (bf16, register
+  // token fragments, no slot on the tensor-core path).  Under stage timing its event pair is the
+  // gate stage's, and the selection and up/down stages are empty.
+  const bool fused = dt == 0 && !dense && h->fused && moe::layer_available(h->ls);
   if (e == cudaSuccess) e = moe::launch_router(p, dt, st);
   if (e == cudaSuccess && tm) e = cudaEventRecord(ev[1], st);
-  if (e == cudaSuccess) e = moe::launch_gate(p, dt, h->ls, st, pdl);
-  if (e == cudaSuccess && dense) e = moe::launch_dense(p, h->ls, 0, st, pdl);
-  if (e == cudaSuccess && tm) e = cudaEventRecord(ev[2], st);
-  if (e == cudaSuccess) e = moe::launch_select(p, h->ls, st, pdl);
-  if (e == cudaSuccess && tm) e = cudaEventRecord(ev[3], st);
-  if (e == cudaSuccess && dense) e = moe::launch_dense(p, h->ls, 1, st, pdl);
-  if (e == cudaSuccess) e = moe::launch_updown(p, dt, h->ls, st, pdl);
-  if (e == cudaSuccess && tm) e = cudaEventRecord(ev[4], st);
+  if (fused) {
+    if (e == cudaSuccess) e = moe::launch_layer(p, h->ls, st, pdl);
+    for (int k = 2; k <= 4 && tm && e == cudaSuccess; ++k) e = cudaEventRecord(ev[k], st);
+  } else {
+    if (e == cudaSuccess) e = moe::launch_gate(p, dt, h->ls, st, pdl);
+    if (e == cudaSuccess && dense) e = moe::launch_dense(p, h->ls, 0, st, pdl);
+    if (e == cudaSuccess && tm) e = cudaEventRecord(ev[2], st);
+    if (e == cudaSuccess) e = moe::launch_select(p, h->ls, st, pdl);
+    if (e == cudaSuccess && tm) e = cudaEventRecord(ev[3], st);
+    if (e == cudaSuccess && dense) e = moe::launch_dense(p, h->ls, 1, st, pdl);
+    if (e == cudaSuccess) e = moe::launch_updown(p, dt, h->ls, st, pdl);
+    if (e == cudaSuccess && tm) e = cudaEventRecord(ev[4], st);
+  }
   // a partial output stays fp32: the sum over the handles is cast once (moe_cast_output)
   if (e == cudaSuccess) e = moe::launch_finalize(p, partial ? 1 : dt, h->ls, st, pdl);
   if (e == cudaSuccess && tm) e = cudaEventRecord(ev[5], st);
@@ -293,8 +308,9 @@ moe_status forward_impl(moe_handle* h, const void* x, int n_tokens, const void* 
     return MOE_ERR_CUDA;
   }
   h->last_tokens = n_tokens;
-  // + gather and three GEMMs on the tensor-core path, + the roster bias kernel
-  h->last_launches = (dense ? 9 : 5) + (roster ? 1 : 0);
+  // router, fused layer, finalize; or the chain of five (+ gather and three GEMMs on the
+  // tensor-core path); + the roster bias kernel
+  h->last_launches = (fused ? 3 : dense ? 9 : 5) + (roster ? 1 : 0);
   return MOE_OK;
 }
 
@@ -342,7 +358,8 @@ moe_status moe_create(const moe_config* cfg, moe_handle** out) {
   cudaError_t e;
   {
     std::lock_guard<std::mutex> lock(moe::setup_mutex());
-    e = moe::configure_kernels(cfg->dtype == MOE_BF16 ? 0 : 1, h->imax, cfg->n_routed,
+    e = moe::configure_kernels(cfg->dtype == MOE_BF16 ? 0 : 1, h->imax,
+                               cfg->n_routed + cfg->n_shared,
                                cfg->max_tokens, cfg->hidden, &h->ls);
   }
   if (e != cudaSuccess) {
@@ -356,6 +373,7 @@ moe_status moe_create(const moe_config* cfg, moe_handle** out) {
     return MOE_ERR_OOM;
   }
   h->dense_min = MOE_DENSE_AUTO;
+  h->fused = true;
   h->e_begin = 0;
   h->e_end = cfg->n_routed;
   h->shared_mask = (1u << cfg->n_shared) - 1u;
@@ -581,6 +599,12 @@ moe_status moe_last_launches(moe_handle* h, int* n) {
 moe_status moe_set_dense_min_tokens(moe_handle* h, int min_tokens) {
   if (!h || min_tokens < MOE_DENSE_AUTO) return MOE_ERR_INVALID_ARG;
   h->dense_min = min_tokens;
+  return MOE_OK;
+}
+
+moe_status moe_set_fused(moe_handle* h, int enable) {
+  if (!h || (enable != 0 && enable != 1)) return MOE_ERR_INVALID_ARG;
+  h->fused = enable != 0;
   return MOE_OK;
 }
 

@@ -9,8 +9,8 @@ import torch
 import synth
 
 from . import (expert_weights, make_config, moe_create, moe_debug_lists, moe_destroy,
-               moe_forward, moe_forward_roster, moe_last_launches, moe_pack_experts, roster,
-               sparsity)
+               moe_forward, moe_forward_roster, moe_last_launches, moe_pack_experts,
+               moe_set_fused, roster, sparsity)
 
 
 class DeviceLayer:
@@ -96,6 +96,10 @@ class DeviceLayer:
                         r["act"])
         torch.cuda.synchronize()
         return r
+
+    def set_fused(self, enable):
+        """Fused layer kernel where it applies (True, the default) or the launch chain."""
+        moe_set_fused(self.h, 1 if enable else 0)
 
     def last_launches(self):
         return moe_last_launches(self.h)

@@ -86,6 +86,7 @@ def test_forward_rejects_null_handle(lib):
     assert lib.moe_debug_lists(None, 1, None, None, None, None, None, None, None) == \
         moe.MOE_ERR_INVALID_ARG
     assert lib.moe_set_dense_min_tokens(None, 8) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_set_fused(None, 1) == moe.MOE_ERR_INVALID_ARG
     assert lib.moe_debug_force_timeout(None, None) == moe.MOE_ERR_INVALID_ARG
     n = ctypes.c_int(-1)
     assert lib.moe_last_launches(None, ctypes.byref(n)) == moe.MOE_ERR_INVALID_ARG
