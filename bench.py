@@ -83,9 +83,10 @@ def parse():
                          "keep the same kernels and per-item work with less memory resident")
     ap.add_argument("--dense-min", type=int, default=DEFAULT_DENSE_MIN,
                     help="path choice for --profile (see moe_set_dense_min_tokens)")
-    ap.add_argument("--no-fused", dest="fused", action="store_false", default=True,
-                    help="run the chain of separate kernels instead of the fused layer kernel "
+    ap.add_argument("--fused", dest="fused", action="store_true", default=False,
+                    help="run the fused layer kernel instead of the chain of separate kernels "
                          "(see moe_set_fused)")
+    ap.add_argument("--no-fused", dest="fused", action="store_false")
     return ap.parse_args()
 
 

@@ -232,12 +232,14 @@ moe_status moe_debug_force_timeout(moe_handle* h, void* stream);
 moe_status moe_set_dense_min_tokens(moe_handle* h, int min_tokens);
 
 /* Fused layer kernel ("Uncovering Intra-expert Activation Sparsity ...", technical summary, Key
- * contributions: the layer stays one fused, graph-capturable unit).  enable = 1 (the default):
- * a bf16 call whose slots all take the sparse kernels, on a hidden size with register token
- * fragments (512, 2048, 2880, 5120), runs gate, selection and up/down as one persistent kernel
- * between the router and the output cast (3 launches instead of 5): a token tile's selections
- * start as soon as its gate rows are done and an expert's up/down as soon as its union is known.
- * enable = 0: always the chain of separate kernels.  The results are the same within rounding of
+ * contributions: the layer stays one fused, graph-capturable unit).  enable = 1: a bf16 call
+ * whose slots all take the sparse kernels, on a hidden size with register token fragments (512,
+ * 2048, 2880, 5120), runs gate, selection and up/down as one persistent kernel between the router
+ * and the output cast (3 launches instead of 5): a token tile's selections start as soon as its
+ * gate rows are done and an expert's up/down as soon as its union is known.  enable = 0 (the
+ * default): the chain of separate kernels, which measured faster on B200 at every batch size
+ * tried (the selections cost the fused kernel's consumer warps as much time as the separate
+ * selection kernel costs the chain, and the last slots' selections stay on its critical path).  The results are the same within rounding of
  * the fp32 output sums (the up/down runs accumulate in another grouping); routing and kept sets
  * are identical.  Under stage timing (moe_profile_stages) the fused kernel's duration is the
  * gate stage's, and the selection and up/down stages are empty.  INVALID_ARG for a

@@ -260,7 +260,7 @@ def moe_set_dense_min_tokens(h, min_tokens):
 
 
 def moe_set_fused(h, enable):
-    """1: gate, selection and up/down as one fused kernel where it applies (the default); 0: the
+    """1: gate, selection and up/down as one fused kernel where it applies; 0 (the default): the
     chain of separate kernels (see include/moe.h)."""
     _check(_lib().moe_set_fused(ctypes.c_void_p(h) if h else None, int(enable)), "moe_set_fused")
 

@@ -40,7 +40,7 @@ constexpr int kCoefWarps = 2;
 constexpr int kLayerThreads = kThreads + 64 + 32 * kCoefWarps;
 constexpr int kCopier = kWarps, kMetaWarp = kWarps + 1, kCoefWarp0 = kWarps + 2;
 constexpr int kGateChunk = 2;  // gate items claimed at a time from the work counter
-constexpr int kGateRun = 8;    // consecutive gate items of a CTA's static rounds
+constexpr int kGateRun = 16;   // consecutive gate items of a CTA's static rounds
 // Records in flight per CTA: the meta warp publishes up to kLayerRing - 1 records ahead of the
 // consumers (record i reuses the slot of record i - kLayerRing once that one is finished).
 constexpr int kLayerRing = 6;
@@ -53,7 +53,8 @@ struct LayerMeta {
   int type;                   // kRecG, kRecU, kRecS
   int end;                    // 1: no more records (the CTA's loops end here)
   int key;                    // token tile id of G and U records (-1 for S)
-  int xlast;                  // U: the CTA's next up/down record is of another token tile
+  int xlast;                  // G, U: the CTA's next record of this kind is of another tile
+                              // (G: 2 when no gate record follows in this CTA)
   int q0, nt, n0;             // G: first pair of the tile, its tokens, first neuron
   int q;                      // S: the pair
   int j, tt, rg;              // U: slot, token tile, row group
@@ -243,68 +244,14 @@ __global__ void __launch_bounds__(kLayerThreads, 1) layer_kernel(FwdParams p, Ri
       return cb++;
     };
 
-    int mi = 0, si = 0, run_cnt = 0;
-    // A finished run of gate items of one token tile (cnt of them, the last one record R) is
-    // added to the tile's counter; the report that completes the count makes the tile's pairs
-    // selection tasks.
-    auto report = [&](const LayerMeta& R, int cnt) {
-      const int I = R.q0 >= p.B * p.k ? p.Ish : p.I;
-      int fire = 0;
-      unsigned k0 = 0;
-      if (lane == 0) {
-        __threadfence();  // the consumers' activations and histogram counts before the count
-        const unsigned old = atomicAdd(&p.tile_done[R.q0], (unsigned)cnt);
-        if (old + (unsigned)cnt == (unsigned)(I / kTileRows)) {
-          __threadfence();
-          k0 = atomicAdd(&p.fq[0], (unsigned)R.nt);
-          fire = 1;
-        }
-      }
-      fire = __shfl_sync(0xffffffffu, fire, 0);
-      k0 = __shfl_sync(0xffffffffu, k0, 0);
-      if (fire && lane < R.nt) {
-        __threadfence();
-        *reinterpret_cast<volatile int*>(&p.s_task[k0 + lane]) = R.q0 + lane + 1;
-      }
-    };
-    // Record r is finished (consumers and copier): a gate record extends its tile's run, which
-    // ends where the next record is not a gate item of the same tile (or nothing follows).
-    auto complete = [&](int r) {
-      const LayerMeta& R = s_meta[r % kLayerRing];
-      if (R.type != kRecG) return;
-      ++run_cnt;
-      int nk = -1;
-      if (r + 1 < mi) {
-        const LayerMeta& N = s_meta[(r + 1) % kLayerRing];
-        if (N.type == kRecG) nk = N.key;
-      }
-      if (nk != R.key) {
-        report(R, run_cnt);
-        run_cnt = 0;
-      }
-    };
-    // Takes the finished records below `upto`, in order; waits for the first one if `block`.
-    // False once the CTA aborts.
-    auto drain = [&](int upto, bool block) -> bool {
-      while (si < upto) {
-        const int m = si % kLayerRing;
-        const uint32_t ph = (si / kLayerRing) & 1;
-        int done = 0;
-        if (lane == 0) done = mbar_test(&edone[m], ph);
-        done = __shfl_sync(0xffffffffu, done, 0);
-        if (!done) {
-          if (!block) return true;
-          if (!mbar_wait(&edone[m], ph, abort, p.err)) return false;
-        }
-        complete(si);
-        ++si;
-      }
-      return true;
-    };
-    // Frees the ring slot of record mi (its record mi - kLayerRing is finished).
+    int mi = 0, si = 0;
+    // Frees the ring slot of record mi: waits until record mi - kLayerRing is finished
+    // (consumers and copier).  False once the CTA aborts.
     auto slot_free = [&]() -> bool {
-      if (!drain(mi - (kLayerRing - 1), true)) return false;
-      return drain(mi - 1, false);
+      for (; si <= mi - kLayerRing; ++si)
+        if (!mbar_wait(&edone[si % kLayerRing], (si / kLayerRing) & 1, abort, p.err))
+          return false;
+      return true;
     };
     auto post = [&](int m) {  // the meta warp's arrivals for a written record
       __syncwarp();
@@ -427,16 +374,48 @@ __global__ void __launch_bounds__(kLayerThreads, 1) layer_kernel(FwdParams p, Ri
     };
     unsigned long long t_wait = 0, t_idle = 0;
     int n_s = 0, n_u = 0;
+    // A gate item's slot entry, local index and token tile (shared items carry the local shared
+    // expert's entry directly)
+    struct GPlace {
+      int4 sl;
+      int local, key;
+    };
+    auto place_g = [&](int item) -> GPlace {
+      GPlace g;
+      if (item < n_pre) {
+        const int o = item / (sh_groups * Bt);  // o-th shared expert of this handle
+        unsigned msk = p.shared_mask;
+        for (int i = 0; i < o; ++i) msk &= msk - 1;
+        const int s_i = __ffs(msk) - 1;
+        g.sl = make_int4(s_i | (1 << 16), p.B, p.B * p.k + s_i * p.B, 0);
+        g.local = item - o * sh_groups * Bt;
+        g.key = (1 << 20) + s_i * 1024 + g.local / sh_groups;
+      } else {
+        const int r = item - n_pre;
+        const int j = find_item_slot(s_tab, n_slots, r);
+        g.sl = s_tab[j];
+        g.local = r - g.sl.w;
+        g.key = j * 1024 + g.local / (p.I / kTileRows);
+      }
+      return g;
+    };
+    // the current gate item and the next one, claimed ahead: a record whose successor is of
+    // another token tile (or none) ends its run, which its consumers then report
     int gcur = claim_g();
+    GPlace gpl = gcur >= 0 ? place_g(gcur) : GPlace{};
+    int gnxt = gcur >= 0 ? claim_g() : -1;
+    GPlace npl = gnxt >= 0 ? place_g(gnxt) : GPlace{};
     int tok_key = -2, tok_l = -1;  // token of lane l in the last gate tile the warp looked up
     unsigned long long idle_t0 = 0;
     bool g_end_seen = false;
+    unsigned sa_next = 0, sc_next = 0;
     while (!*abort) {
-      // the task counters are read before the wait for a free record, which hides their latency
-      unsigned sa = 0, sc = 0;
-      if (lane == 0 && routed_known && pend_s == -1) {
-        sa = ld_volatile(&p.fq[0]);
-        sc = ld_volatile(&p.fq[1]);
+      // the task counters as lane 0 read them in the previous iteration (the loads of the next
+      // iteration's values are issued here, so their round trip overlaps this one)
+      const unsigned sa = sa_next, sc = sc_next;
+      if (lane == 0 && routed_known) {
+        sa_next = ld_volatile(&p.fq[0]);
+        sc_next = ld_volatile(&p.fq[1]);
       }
       {
         const unsigned long long t0 = p.trace ? globaltimer() : 0ull;
@@ -461,25 +440,8 @@ __global__ void __launch_bounds__(kLayerThreads, 1) layer_kernel(FwdParams p, Ri
         continue;
       }
       if (gcur >= 0) {
-        // gate item gcur: its slot entry and local index (shared items carry the local shared
-        // expert's entry directly)
-        int4 sl;
-        int local, key;
-        if (gcur < n_pre) {
-          const int o = gcur / (sh_groups * Bt);  // o-th shared expert of this handle
-          unsigned msk = p.shared_mask;
-          for (int i = 0; i < o; ++i) msk &= msk - 1;
-          const int s_i = __ffs(msk) - 1;
-          sl = make_int4(s_i | (1 << 16), p.B, p.B * p.k + s_i * p.B, 0);
-          local = gcur - o * sh_groups * Bt;
-          key = (1 << 20) + s_i * 1024 + local / sh_groups;
-        } else {
-          const int r = gcur - n_pre;
-          const int j = find_item_slot(s_tab, n_slots, r);
-          sl = s_tab[j];
-          local = r - sl.w;
-          key = j * 1024 + local / (p.I / kTileRows);
-        }
+        const int4 sl = gpl.sl;
+        const int local = gpl.local, key = gpl.key;
         const int kind = sl.x >> 16, ex = sl.x & 0xffff, T = sl.y, q0 = sl.z;
         const int I = kind ? p.Ish : p.I;
         const int tt = local / (I / kTileRows), rg = local % (I / kTileRows);
@@ -492,6 +454,9 @@ __global__ void __launch_bounds__(kLayerThreads, 1) layer_kernel(FwdParams p, Ri
           s_meta[m].type = kRecG;
           s_meta[m].end = 0;
           s_meta[m].key = key;
+          // 2: the run ends and no gate record follows in this CTA (its report is settled at
+          // once: nothing later would look at it)
+          s_meta[m].xlast = gnxt < 0 ? 2 : npl.key != key ? 1 : 0;
           s_meta[m].q0 = q0 + tt * kTileTok;
           s_meta[m].nt = nt;
           s_meta[m].n0 = rg * kTileRows;
@@ -514,7 +479,10 @@ __global__ void __launch_bounds__(kLayerThreads, 1) layer_kernel(FwdParams p, Ri
         if (lane == 0) mbar_arrive(&mfull[m]);
         __syncwarp();
         ++mi;
-        gcur = claim_g();
+        gcur = gnxt;
+        gpl = npl;
+        gnxt = gcur >= 0 ? claim_g() : -1;
+        if (gnxt >= 0) npl = place_g(gnxt);
         idle_t0 = 0;
         continue;
       }
@@ -554,9 +522,8 @@ __global__ void __launch_bounds__(kLayerThreads, 1) layer_kernel(FwdParams p, Ri
         idle_t0 = 0;
         continue;
       }
-      if (routed_known && u_done && si == mi) break;
-      // nothing to publish: finish the records in flight (a run that ends here is reported)
-      if (!drain(mi, false)) break;
+      if (routed_known && u_done) break;
+      // nothing to publish yet
       const unsigned long long now = globaltimer();
       if (idle_t0 == 0) idle_t0 = now;
       if (now - idle_t0 > kWaitLimitNs) {
@@ -714,6 +681,10 @@ __global__ void __launch_bounds__(kLayerThreads, 1) layer_kernel(FwdParams p, Ri
   uint4 xr[NK][BPW];
   int it = 0, ib = 0, cur = -1;
   int run_key = -1;  // token tile of the open run of up/down sums in tensor memory
+  int g_run = 0;     // thread 0: gate records of the current run of one token tile
+  // thread 0: the last run report, whose result is looked at one gate record later
+  int rep_q0 = -1, rep_cnt = 0, rep_nt = 0;
+  unsigned rep_old = 0, rep_target = 0;
   bool nan_seen = false, waited = false;
   const int nblk = rc.kc / 32, nsub = rc.kc / 64;
   const uint32_t tmem_warp = tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + 256u * (warp >> 2);
@@ -728,6 +699,15 @@ __global__ void __launch_bounds__(kLayerThreads, 1) layer_kernel(FwdParams p, Ri
     if (mi == 0) trace_point(p.trace, 1, 2);
     const LayerMeta& mt = s_meta[m];
     const int type = mt.type;
+    if (type != kRecG && threadIdx.x == 0 && rep_q0 >= 0) {  // a pending run report
+      if (rep_old + (unsigned)rep_cnt == rep_target && !*abort) {
+        __threadfence();
+        const unsigned k0 = atomicAdd(&p.fq[0], (unsigned)rep_nt);
+        for (int i = 0; i < rep_nt; ++i)
+          *reinterpret_cast<volatile int*>(&p.s_task[k0 + i]) = rep_q0 + i + 1;
+      }
+      rep_q0 = -1;
+    }
     if (type == kRecS) {
       // ---- selection of pair mt.q; the CTA that completes the slot's union publishes it
       if (!waited) {
@@ -814,8 +794,44 @@ __global__ void __launch_bounds__(kLayerThreads, 1) layer_kernel(FwdParams p, Ri
             if (uses_hist(p, q0 >= p.B * p.k)) hist_add(p, q0 + ti, a);
           }
         }
-        asm volatile("bar.sync 3, 128;" ::: "memory");
-        if (threadIdx.x == 0) {  // both arrivals on mfull precede the record's release
+        if (xlast) asm volatile("bar.sync 3, 128;" ::: "memory");  // the run's last stores
+        if (threadIdx.x == 0) {
+          // A pending report (of an earlier run) is checked first: its round trip overlapped
+          // the records since.  The report that completes a tile's count makes the tile's pairs
+          // selection tasks.
+          if (rep_q0 >= 0) {
+            if (rep_old + (unsigned)rep_cnt == rep_target && !aborted) {
+              __threadfence();
+              const unsigned k0 = atomicAdd(&p.fq[0], (unsigned)rep_nt);
+              for (int i = 0; i < rep_nt; ++i)
+                *reinterpret_cast<volatile int*>(&p.s_task[k0 + i]) = rep_q0 + i + 1;
+            }
+            rep_q0 = -1;
+          }
+          // The run of gate records of this token tile ends here: its count goes to the tile's
+          // counter, after a fence that makes these records' activations and histogram counts
+          // visible.
+          ++g_run;
+          if (xlast) {
+            const int I = q0 >= p.B * p.k ? p.Ish : p.I;
+            __threadfence();
+            rep_old = atomicAdd(&p.tile_done[q0], (unsigned)g_run);
+            rep_cnt = g_run;
+            rep_target = (unsigned)(I / kTileRows);
+            rep_q0 = q0;
+            rep_nt = nt;
+            g_run = 0;
+            if (xlast == 2) {
+              if (rep_old + (unsigned)rep_cnt == rep_target && !aborted) {
+                __threadfence();
+                const unsigned k0 = atomicAdd(&p.fq[0], (unsigned)rep_nt);
+                for (int i = 0; i < rep_nt; ++i)
+                  *reinterpret_cast<volatile int*>(&p.s_task[k0 + i]) = rep_q0 + i + 1;
+              }
+              rep_q0 = -1;
+            }
+          }
+          // both arrivals on mfull precede the record's release
           mbar_wait(&mfull[m], ph, abort, p.err);
           mbar_arrive(&edone[m]);
         }

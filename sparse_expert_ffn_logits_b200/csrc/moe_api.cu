@@ -48,7 +48,7 @@ struct moe_handle {
   float* roster_bias;  // device [max_tokens][E]: the roster bias of the current call
   int e_begin, e_end;     // routed experts this handle evaluates (all by default)
   unsigned shared_mask;   // shared experts this handle evaluates (all by default)
-  bool fused;             // the fused layer kernel where it applies (default on)
+  bool fused;             // the fused layer kernel where it applies (default off)
 };
 
 namespace {
@@ -373,7 +373,7 @@ moe_status moe_create(const moe_config* cfg, moe_handle** out) {
     return MOE_ERR_OOM;
   }
   h->dense_min = MOE_DENSE_AUTO;
-  h->fused = true;
+  h->fused = false;
   h->e_begin = 0;
   h->e_end = cfg->n_routed;
   h->shared_mask = (1u << cfg->n_shared) - 1u;

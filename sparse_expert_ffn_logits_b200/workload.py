@@ -98,7 +98,7 @@ class DeviceLayer:
         return r
 
     def set_fused(self, enable):
-        """Fused layer kernel where it applies (True, the default) or the launch chain."""
+        """Fused layer kernel where it applies (True) or the launch chain (False, the default)."""
         moe_set_fused(self.h, 1 if enable else 0)
 
     def last_launches(self):

@@ -42,9 +42,8 @@ def test_roster_steps_match_the_oracle(shape, m, delta):
             rep = parity.compare(dl, xh, xd, ("topk", 0.5), rule_s, router_bias=bias,
                                  expert_cache=cache, shared_weights=shared,
                                  name=f"{shape.name} roster step {step}")
-            # roster bias, router, then the fused layer kernel (bf16) or the chain of three
-            # (fp32), and the output cast
-            assert moe_last_launches(dl.h) == (4 if shape.dtype == "bf16" else 6)
+            # roster bias, router, gate, selection, up/down, output cast
+            assert moe_last_launches(dl.h) == 6
             oracle.roster_update(counts_h, rep.idx)
             assert np.array_equal(counts_d.cpu().numpy(), counts_h), f"counts differ at {step}"
             for t in range(B):
