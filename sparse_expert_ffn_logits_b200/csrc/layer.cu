@@ -40,7 +40,7 @@ constexpr int kCoefWarps = 2;
 constexpr int kLayerThreads = kThreads + 64 + 32 * kCoefWarps;
 constexpr int kCopier = kWarps, kMetaWarp = kWarps + 1, kCoefWarp0 = kWarps + 2;
 constexpr int kGateChunk = 2;  // gate items claimed at a time from the work counter
-constexpr int kGateRun = 16;   // consecutive gate items of a CTA's static rounds
+constexpr int kGateRun = 8;    // consecutive gate items of a CTA's static rounds
 // Records in flight per CTA: the meta warp publishes up to kLayerRing - 1 records ahead of the
 // consumers (record i reuses the slot of record i - kLayerRing once that one is finished).
 constexpr int kLayerRing = 6;
