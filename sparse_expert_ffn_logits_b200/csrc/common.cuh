@@ -15,6 +15,13 @@ constexpr int kMaxTopK = 16;
 constexpr int kMaxShared = 8;
 constexpr int kMaxRouted = 512;
 constexpr int kMaxTokens = 1024;
+// A sparse shared expert evaluates every token; up to kMaxSharedTiles token tiles (64 tokens)
+// each of its tiles is a slot of its own, with its own union of kept neurons (the up/down rows
+// a tile reads are those its own tokens keep).  Slot table capacity: routed experts + shared
+// experts' tiles.
+constexpr int kMaxSharedTiles = 8;
+constexpr int kMaxSlots = kMaxRouted + kMaxShared * kMaxSharedTiles;
+__host__ __device__ constexpr int slot_capacity(int E, int S) { return E + S * kMaxSharedTiles; }
 constexpr int kMaxHsplit = 16;     // router slices of H
 constexpr int kMaxI = 16384;       // largest intermediate size
 
@@ -89,16 +96,16 @@ struct FwdParams {
   int* pair_token;     // [Pmax]
   float* pair_w;       // [Pmax]
   int* pair_slot;      // [Pmax]
-  Slot* slots;         // [E+S]
+  Slot* slots;         // [slot_capacity(E, S)]
   int* meta;           // [kMetaWords]
   unsigned* tile_ticket;   // [ceil(Bmax/8)]
   unsigned* global_ticket; // [1]
-  unsigned* slot_ticket;   // [E+S]
+  unsigned* slot_ticket;   // [slot_capacity(E, S)]
   float* act;          // [Pmax][Imax]
   uint32_t* maskbits;  // [Pmax][Imax/32]
-  uint32_t* ubits;     // [E+S][Imax/32]
-  int* ulist;          // [E+S][Imax] ascending union rows of each slot
-  int* ucnt;           // [E+S]
+  uint32_t* ubits;     // [slot_capacity(E, S)][Imax/32]
+  int* ulist;          // [slot_capacity(E, S)][Imax] ascending union rows of each slot
+  int* ucnt;           // [slot_capacity(E, S)]
   float* out_acc;      // [Bmax][H]
   int* err;            // device error word
   const void* zero_row;  // H zero elements (source of the copies of absent tokens)
@@ -119,7 +126,7 @@ struct FwdParams {
   int* s_task;                // [Pmax] selection tasks in the order they became ready: pair + 1
   unsigned* fq;               // [4] selection tasks reserved, claimed; up/down items claimed
   unsigned long long* u_res;  // [1] up/down entries published << 32 | up/down items reserved
-  int4* u_ent;                // [E+S] per entry: {slot + 1, first item, items, union rows}
+  int4* u_ent;                // [slot_capacity(E, S)] per entry: {slot + 1, first item, items, union rows}
 };
 
 // Phase timestamps for tracing: kernel k, CTA b, point i (i < kTracePoints).

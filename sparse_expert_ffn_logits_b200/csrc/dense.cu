@@ -40,7 +40,6 @@ constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kDenseThreads = 192;
 constexpr int kProducerWarp = 4, kMmaWarp = 5;
 constexpr int kTmemCols = 512;             // two accumulators of 256 fp32 columns
-constexpr int kMaxSlots = kMaxRouted + kMaxShared;
 constexpr int kDenseSmem = kStages * kStageBytes + 1024;  // + alignment slack
 
 // ---- tcgen05 / TMA primitives -----------------------------------------------------------------
@@ -160,7 +159,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
   // tile table over the dense slots (every slot entry that can exist is read speculatively)
   {
     const int n_slots = ld_cg(&p.meta[kMetaSlots]);
-    const int n_max = min(p.E + p.S, kMaxSlots);
+    const int n_max = min(slot_capacity(p.E, p.S), kMaxSlots);
     const int per = (n_max + blockDim.x - 1) / blockDim.x;
     const int b0 = min(n_max, (int)threadIdx.x * per), b1 = min(n_max, b0 + per);
     int c = 0;
@@ -187,7 +186,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
   __syncthreads();
   tc_fence_after();
   const int n_tiles = s_total;
-  const int n_max = min(p.E + p.S, kMaxSlots);
+  const int n_max = min(slot_capacity(p.E, p.S), kMaxSlots);
   const uint32_t tmem_base = s_tmem;
   auto tile_at = [&](int t) -> TileRef {
     TileRef r;

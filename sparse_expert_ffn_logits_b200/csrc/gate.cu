@@ -31,7 +31,6 @@
 namespace moe {
 namespace {
 
-constexpr int kMaxSlots = kMaxRouted + kMaxShared;
 constexpr int kRingThreads = kThreads + 64;  // 8 consumer warps, copier, meta
 constexpr int kCopier = kWarps, kMetaWarp = kWarps + 1;
 
@@ -118,7 +117,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) gate_tma_kernel(FwdParams p, 
       // at n_slots and beyond are stale and never searched
       n_slots = ld_cg(&p.meta[kMetaSlots]);
       const int n_routed = ld_cg(&p.meta[kMetaGateItems]) - n_pre;
-      for (int j = lane; j < min(p.E + p.S, kMaxSlots); j += 32) {
+      for (int j = lane; j < min(slot_capacity(p.E, p.S), kMaxSlots); j += 32) {
         const Slot sl = load_slot(&p.slots[j]);
         s_tab[j] = make_int4(sl.expert | (sl.kind << 16), sl.T, sl.q0, sl.item0);
       }

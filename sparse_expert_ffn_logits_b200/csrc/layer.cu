@@ -35,7 +35,6 @@
 namespace moe {
 namespace {
 
-constexpr int kMaxSlots = kMaxRouted + kMaxShared;
 constexpr int kCoefWarps = 2;
 constexpr int kLayerThreads = kThreads + 64 + 32 * kCoefWarps;
 constexpr int kCopier = kWarps, kMetaWarp = kWarps + 1, kCoefWarp0 = kWarps + 2;
@@ -126,7 +125,7 @@ __global__ void __launch_bounds__(kLayerThreads, 1) layer_kernel(FwdParams p, Ri
   __shared__ SelShared<kThreads> s_sel;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
-  const int n_slot_max = min(p.E + p.S, kMaxSlots);
+  const int n_slot_max = min(slot_capacity(p.E, p.S), kMaxSlots);
   const LayerSmem L = layer_smem(n_slot_max);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + rc.ns;

@@ -26,7 +26,8 @@ __global__ void finalize_kernel(FwdParams p) {
     p.tile_done[i] = 0;
     p.s_task[i] = 0;
   }
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.E + p.S; i += gridDim.x * blockDim.x)
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < slot_capacity(p.E, p.S);
+       i += gridDim.x * blockDim.x)
     p.u_ent[i] = make_int4(0, 0, 0, 0);
   if (blockIdx.x == 0 && threadIdx.x < 4) p.fq[threadIdx.x] = 0;
   if (blockIdx.x == 0 && threadIdx.x == 0) *p.u_res = 0ull;

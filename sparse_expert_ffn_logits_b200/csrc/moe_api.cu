@@ -161,7 +161,8 @@ struct Carve {
 size_t carve(moe_handle* h, char* base) {
   const moe_config& c = h->cfg;
   const size_t Bm = (size_t)c.max_tokens, E = c.n_routed, k = c.top_k, S = c.n_shared;
-  const size_t Pm = Bm * (k + S), Im = h->imax, Wm = Im / 32, slots = E + S;
+  const size_t Pm = Bm * (k + S), Im = h->imax, Wm = Im / 32,
+               slots = (size_t)moe::slot_capacity((int)E, (int)S);
   Carve cv{base, 0};
   FwdParams& p = h->base;
   p.logits = cv.take<float>(Bm * E);
@@ -359,7 +360,7 @@ moe_status moe_create(const moe_config* cfg, moe_handle** out) {
   {
     std::lock_guard<std::mutex> lock(moe::setup_mutex());
     e = moe::configure_kernels(cfg->dtype == MOE_BF16 ? 0 : 1, h->imax,
-                               cfg->n_routed + cfg->n_shared,
+                               moe::slot_capacity(cfg->n_routed, cfg->n_shared),
                                cfg->max_tokens, cfg->hidden, &h->ls);
   }
   if (e != cudaSuccess) {

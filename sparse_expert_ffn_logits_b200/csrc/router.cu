@@ -204,8 +204,13 @@ __device__ void group_pairs(const FwdParams& p, uint32_t* dyn, unsigned long lon
   const int routed_items = (int)(tot >> 32);
   const unsigned smask = p.shared_mask;
   const int n_shared_local = __popc(smask & ((1u << S) - 1u));
-  const int n_slots = n_touched + n_shared_local;
-  const int sh_items = B < p.dense_min ? (p.Ish / kTileRows) * ((B + kTileTok - 1) / kTileTok) : 0;
+  // A sparse shared expert with at most kMaxSharedTiles token tiles has a slot per tile (each
+  // with its own union); otherwise one slot for all B tokens.
+  const int Bt = (B + kTileTok - 1) / kTileTok;
+  const bool split = B < p.dense_min && Bt <= kMaxSharedTiles;
+  const int sh_tiles = split ? Bt : 1;
+  const int n_slots = n_touched + n_shared_local * sh_tiles;
+  const int sh_items = B < p.dense_min ? (p.Ish / kTileRows) * (split ? 1 : Bt) : 0;  // per slot
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     if (cnt[e] > 0 && e >= p.e_begin && e < p.e_end) {
       const unsigned long long pr = pre[e];
@@ -220,18 +225,22 @@ __device__ void group_pairs(const FwdParams& p, uint32_t* dyn, unsigned long lon
       p.slots[(int)((pr >> 20) & 0xFFF)] = s;
     }
   }
-  // local shared expert s_i: slot n_touched + (its rank among the local shared experts)
+  // local shared expert s_i: first slot n_touched + sh_tiles (its rank among the local shared
+  // experts); its tile tt is that slot + tt when split
   auto shared_slot = [&](int s_i) -> int {
-    return ((smask >> s_i) & 1u) ? n_touched + __popc(smask & ((1u << s_i) - 1u)) : -1;
+    return ((smask >> s_i) & 1u) ? n_touched + sh_tiles * __popc(smask & ((1u << s_i) - 1u))
+                                 : -1;
   };
-  for (int s_i = threadIdx.x; s_i < S; s_i += blockDim.x) {
-    const int j = shared_slot(s_i);
-    if (j < 0) continue;
+  for (int i = threadIdx.x; i < S * sh_tiles; i += blockDim.x) {
+    const int s_i = i / sh_tiles, tt = i % sh_tiles;
+    const int j0 = shared_slot(s_i);
+    if (j0 < 0) continue;
+    const int j = j0 + tt;
     Slot s;
     s.kind = 1;
     s.expert = s_i;
-    s.T = B;
-    s.q0 = B * k + s_i * B;
+    s.T = split ? min(kTileTok, B - tt * kTileTok) : B;
+    s.q0 = B * k + s_i * B + tt * kTileTok;
     s.I = p.Ish;
     s.item0 = routed_items + (j - n_touched) * sh_items;
     s.pad0 = s.pad1 = 0;
@@ -258,7 +267,8 @@ __device__ void group_pairs(const FwdParams& p, uint32_t* dyn, unsigned long lon
   for (int i = threadIdx.x; i < B * S; i += blockDim.x) {
     const int s_i = i / B, t = i % B;
     const int q = B * k + s_i * B + t;
-    const int j = shared_slot(s_i);
+    const int j0 = shared_slot(s_i);
+    const int j = j0 < 0 ? -1 : j0 + (split ? t / kTileTok : 0);
     p.pair_token[q] = t;
     p.pair_w[q] = 1.0f;
     p.pair_slot[q] = j;
@@ -267,7 +277,7 @@ __device__ void group_pairs(const FwdParams& p, uint32_t* dyn, unsigned long lon
   if (threadIdx.x == 0) {
     p.meta[kMetaSlots] = n_slots;
     p.meta[kMetaPairs] = B * (k + S);
-    p.meta[kMetaGateItems] = routed_items + n_shared_local * sh_items;
+    p.meta[kMetaGateItems] = routed_items + n_shared_local * sh_tiles * sh_items;
     p.meta[kMetaTouched] = n_touched;
   }
 }

@@ -23,7 +23,11 @@ __global__ void __launch_bounds__(NT) select_kernel(FwdParams p) {
   auto bar = []() { __syncthreads(); };
   for (int q = blockIdx.x; q < n_pairs; q += gridDim.x) {
     int j;
-    select_pair<NT, false>(p, q, (int)threadIdx.x, sm, ss, bar, nan_seen, &j);
+    const bool first = q == (int)blockIdx.x;
+    auto mark = [&](int i) {
+      if (first) trace_point(p.trace, 2, i);
+    };
+    select_pair<NT, false>(p, q, (int)threadIdx.x, sm, ss, bar, nan_seen, &j, mark);
   }
   if (nan_seen) set_error(p.err, kErrNanAct);
   trace_point(p.trace, 2, 7);

@@ -75,9 +75,15 @@ __host__ __device__ constexpr size_t sel_key_bytes(int imax) {
 // are turned into keys in place.  Returns the slot j of the pair in *slot_out, and the union size
 // when this call compacted the slot's union (the slot's last pair), else -1.  A pair of no slot
 // (another handle's expert) does nothing and returns -1 with *slot_out = -1.
-template <int NT, bool kStaged, typename Bar>
+struct NoMark {
+  __device__ __forceinline__ void operator()(int) const {}
+};
+
+// mark(i) is called by every thread at the phase boundaries i = 2 (keys in place), 3 (cut
+// found), 4 (kept masks stored), 5 (union bits fenced), 6 (ticket taken), for tracing.
+template <int NT, bool kStaged, typename Bar, typename Mark = NoMark>
 __device__ int select_pair(const FwdParams& p, int q, int tid, uint32_t* key, SelShared<NT>& ss,
-                           Bar bar, bool& nan_seen, int* slot_out) {
+                           Bar bar, bool& nan_seen, int* slot_out, Mark mark = Mark{}) {
   constexpr int kSelThreads = NT, kSelWarps = NT / 32;
   constexpr int kBpt = kHistBins / NT;  // histogram bins per thread (8 or 2)
   static_assert(kBpt == 8 || kBpt == 2, "histogram bins per thread");
@@ -118,6 +124,9 @@ __device__ int select_pair(const FwdParams& p, int q, int tid, uint32_t* key, Se
   const int j = __ldcg(&p.pair_slot[q]);  // the expert's slot, for its union row
   *slot_out = j;
   if (j < 0) return -1;  // an expert another handle evaluates (the same for all NT threads)
+  // A slot with one pair: the pair's kept set is the union, compacted straight from the masks in
+  // shared memory (no union bitmask, no fence, no ticket).
+  const bool single = __ldcg(&p.slots[j].T) == 1;
   if (tid == 0) ss.ncand = 0;
   if constexpr (kStaged) {
     for (int n = tid; n < I; n += kSelThreads) {
@@ -152,6 +161,7 @@ __device__ int select_pair(const FwdParams& p, int q, int tid, uint32_t* key, Se
     }
   }
   bar();
+  mark(2);
   const int mode = p.sel_mode[kind];
   const int K = min(p.sel_K[kind], I);
   const float thr = p.sel_t[kind];
@@ -206,18 +216,24 @@ __device__ int select_pair(const FwdParams& p, int q, int tid, uint32_t* key, Se
     if (gathered) {
       if (tid == 0) ss.nset = 0;
       bar();
-      for (int n0 = warp * 32; n0 < I; n0 += kSelThreads) {  // warp-aggregated appends
+      // each warp counts its hits over its chunks, reserves its range with one atomic, then
+      // writes the keys in chunk order (the keys are read twice from shared memory)
+      int whits = 0;
+      for (int n0 = warp * 32; n0 < I; n0 += kSelThreads) {
+        const int n = n0 + lane;
+        whits += __popc(__ballot_sync(0xffffffffu, n < I && (key[n] & pmask) == prefix));
+      }
+      int base = 0;
+      if (lane == 0 && whits) base = atomicAdd(&ss.nset, whits);
+      base = __shfl_sync(0xffffffffu, base, 0);
+      for (int n0 = warp * 32; n0 < I && whits; n0 += kSelThreads) {
         const int n = n0 + lane;
         const uint32_t u = n < I ? key[n] : 0u;
         const bool hit = n < I && (u & pmask) == prefix;
         const unsigned hm = __ballot_sync(0xffffffffu, hit);
-        if (hm) {
-          int base = 0;
-          if (lane == 0) base = atomicAdd(&ss.nset, __popc(hm));
-          base = __shfl_sync(0xffffffffu, base, 0);
-          const int at = base + __popc(hm & lanemask_lt());
-          if (hit && at < kSelThreads) ss.cset[at] = u;  // at < cand <= NT by construction
-        }
+        const int at = base + __popc(hm & lanemask_lt());
+        if (hit && at < kSelThreads) ss.cset[at] = u;  // at < cand <= NT by construction
+        base += __popc(hm);
       }
       bar();
       mine_ok = tid < cand && tid < ss.nset;  // cand == ss.nset by construction
@@ -310,6 +326,7 @@ __device__ int select_pair(const FwdParams& p, int q, int tid, uint32_t* key, Se
       eqtot = ss.eqtot;
     }
   }
+  mark(3);
   // Kept set, one ballot per 32-neuron chunk c (neurons 32c .. 32c + 31), gathered in shared
   // memory, then written by all threads at once as the pair's mask row and OR-ed into the
   // expert's union row.  When every key equal to the cut is kept (the usual case) the mask is
@@ -367,32 +384,44 @@ __device__ int select_pair(const FwdParams& p, int q, int tid, uint32_t* key, Se
   for (int c = tid; c < nch; c += kSelThreads) {
     const uint32_t km = s_km[c];
     mrow[c] = km;
-    if (km) red_or(&urow[c], km);
+    if (km && !single) red_or(&urow[c], km);
   }
-  // the last pair of an expert to finish compacts the expert's union (atomic ticket, no
-  // waiting): every pair's union bits are published before its ticket
-  __threadfence();
-  bar();
-  if (tid == 0) {
-    const unsigned ticket = atomicAdd(&p.slot_ticket[j], 1u);
-    ss.last = ticket == (unsigned)__ldcg(&p.slots[j].T) - 1u;
+  mark(4);
+  if (!single) {
+    // the last pair of an expert to finish compacts the expert's union (atomic ticket, no
+    // waiting): every pair's union bits are published before its ticket
+    __threadfence();
+    bar();
+    mark(5);
+    if (tid == 0) {
+      const unsigned ticket = atomicAdd(&p.slot_ticket[j], 1u);
+      ss.last = ticket == (unsigned)__ldcg(&p.slots[j].T) - 1u;
+    }
+  } else if (tid == 0) {
+    ss.last = 1;
   }
   bar();
+  mark(6);
   int result = -1;
   if (ss.last) {
     // All NT threads compact the union bitmask into the ascending row list and clear it:
     // thread t owns the words [t wpt, (t + 1) wpt), a scan of their bit counts gives each
     // word's first list position, and then each warp writes one word per step, lane l placing
     // bit l at its rank among the word's set bits.
-    __threadfence();
+    if (!single) __threadfence();
     const int W = I / 32, wpt = (W + kSelThreads - 1) / kSelThreads;
     uint32_t* s_word = key;                                // [W] union words (keys are done)
     int* s_base = reinterpret_cast<int*>(key + Imax / 2);  // [W] first position of each word
     const int wb = min(W, tid * wpt), we = min(W, wb + wpt);
     int c = 0;
     for (int w = wb; w < we; ++w) {
-      const uint32_t b = __ldcg(&urow[w]);
-      urow[w] = 0;
+      uint32_t b;
+      if (single) {
+        b = s_km[w];
+      } else {
+        b = __ldcg(&urow[w]);
+        urow[w] = 0;
+      }
       s_word[w] = b;
       c += __popc(b);
     }
@@ -410,7 +439,7 @@ __device__ int select_pair(const FwdParams& p, int q, int tid, uint32_t* key, Se
     }
     if (tid == 0) {
       p.ucnt[j] = total;
-      p.slot_ticket[j] = 0;
+      if (!single) p.slot_ticket[j] = 0;
     }
     result = total;
   }

@@ -24,7 +24,6 @@
 namespace moe {
 namespace {
 
-constexpr int kMaxSlots = kMaxRouted + kMaxShared;
 // 8 consumer warps, the copier, the lead meta warp (token tiles) and kCoefWarps coefficient
 // warps that fill alternate item records in parallel (each record costs two dependent L2 reads)
 constexpr int kCoefWarps = 2;
@@ -156,7 +155,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) updown_tma_kernel(FwdParams p
     // items per slot = ceil(union rows / 16) * token tiles; exclusive prefix into s_tab[].w.
     // Every slot entry that can exist (E + S) is read together with the slot count (one round
     // trip); entries at n_slots and beyond count as empty.
-    const int n_max = min(p.E + p.S, kMaxSlots);
+    const int n_max = min(slot_capacity(p.E, p.S), kMaxSlots);
     const int per = (n_max + blockDim.x - 1) / blockDim.x;
     const int b0 = min(n_max, (int)threadIdx.x * per), b1 = min(n_max, b0 + per);
     int c = 0;
