@@ -92,16 +92,20 @@ __device__ int select_pair(const FwdParams& p, int q, int tid, uint32_t* key, Se
   // The first activations are requested before the pair's slot is known (the row is Imax long
   // whatever the expert's I): one round trip instead of three dependent ones.
   const float4* a4 = reinterpret_cast<const float4*>(p.act + (size_t)q * Imax);
+  // routed pairs come first (B * k of them), then the shared experts' pairs
+  const int kind = q >= p.B * p.k ? 1 : 0;
+  const int I = kind ? p.Ish : p.I;
+  // top-K with K = 0 or K >= I keeps nothing or everything: the scores are not read (the gate
+  // epilogues already flag NaN activations)
+  const bool need_keys = p.sel_mode[kind] == 1 || (p.sel_K[kind] > 0 && p.sel_K[kind] < I);
   constexpr int kKeyLoads = 8;  // 16-byte loads in flight per thread
   float4 f[kKeyLoads];
 #pragma unroll
   for (int u = 0; u < kKeyLoads; ++u) {
     const int v = tid + u * kSelThreads;
-    f[u] = !kStaged && v < Imax / 4 ? __ldcg(a4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+    f[u] = !kStaged && need_keys && v < Imax / 4 ? __ldcg(a4 + v)
+                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  // routed pairs come first (B * k of them), then the shared experts' pairs
-  const int kind = q >= p.B * p.k ? 1 : 0;
-  const int I = kind ? p.Ish : p.I;
   // the pair's score histogram (top-K pairs) is requested together with its activations:
   // thread r holds the kBpt bins counted from the top, [kBpt (NT - 1 - r), kBpt (NT - r))
   const bool hist_on = uses_hist(p, kind);
@@ -125,10 +129,13 @@ __device__ int select_pair(const FwdParams& p, int q, int tid, uint32_t* key, Se
   *slot_out = j;
   if (j < 0) return -1;  // an expert another handle evaluates (the same for all NT threads)
   // A slot with one pair: the pair's kept set is the union, compacted straight from the masks in
-  // shared memory (no union bitmask, no fence, no ticket).
-  const bool single = __ldcg(&p.slots[j].T) == 1;
+  // shared memory (no union bitmask, no fence, no ticket).  A slot on the tensor-core path needs
+  // no union at all: its GEMMs read the mask rows.
+  const int Tj = __ldcg(&p.slots[j].T);
+  const bool single = Tj == 1, no_union = Tj >= p.dense_min;
   if (tid == 0) ss.ncand = 0;
-  if constexpr (kStaged) {
+  if (!need_keys) {
+  } else if constexpr (kStaged) {
     for (int n = tid; n < I; n += kSelThreads) {
       const float a = __uint_as_float(key[n]);
       if (isnan(a)) nan_seen = true;
@@ -339,7 +346,7 @@ __device__ int select_pair(const FwdParams& p, int q, int tid, uint32_t* key, Se
   uint32_t* s_em = s_km + Imax / 32;  // [Imax / 32] tie masks
   if (!radix || eqtot == need) {
     for (int c = warp; c < nch; c += kSelWarps) {
-      const uint32_t u = key[32 * c + lane];
+      const uint32_t u = need_keys ? key[32 * c + lane] : 0u;
       bool k_n;
       if (radix) k_n = u >= tau;
       else if (mode == 1) k_n = __uint_as_float(u) > thr;
@@ -384,9 +391,13 @@ __device__ int select_pair(const FwdParams& p, int q, int tid, uint32_t* key, Se
   for (int c = tid; c < nch; c += kSelThreads) {
     const uint32_t km = s_km[c];
     mrow[c] = km;
-    if (km && !single) red_or(&urow[c], km);
+    if (km && !single && !no_union) red_or(&urow[c], km);
   }
   mark(4);
+  if (no_union) {
+    bar();  // the next pair reuses the key and chunk buffers
+    return -1;
+  }
   if (!single) {
     // the last pair of an expert to finish compacts the expert's union (atomic ticket, no
     // waiting): every pair's union bits are published before its ticket
