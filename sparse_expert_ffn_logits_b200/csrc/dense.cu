@@ -112,10 +112,18 @@ struct DenseMaps {
   CUtensorMap b;         // token rows: xp (gate, up) or hbuf (down)
 };
 
-// Tile t of the launch: slot j, M tile mt, N tile nt (all M tiles of one N tile are consecutive).
+// Tile t of the launch: slot j, M tile mt, N tile nt (all M tiles of one N tile are consecutive),
+// and the range [kb0, kb1) of 64-wide K blocks it contracts (all of them, except for a down
+// GEMM split over K).
 struct TileRef {
-  int j, kind, expert, T, q0, m0, n0, ntok, mext;
+  int j, kind, expert, T, q0, m0, n0, ntok, mext, kb0, kb1;
 };
+
+// Largest K split of the down GEMM.  Its epilogue adds w * D into the output accumulator, so
+// partial sums over K ranges may be added separately.  A down GEMM with fewer tiles than CTAs
+// (a large shared expert alone on this path: H / 128 tiles) is split until its tiles cover the
+// grid.  The gate and up GEMMs are never split: their epilogues are not linear in D.
+constexpr int kMaxKSplit = 4;
 
 template <int kMode>
 __global__ void __launch_bounds__(kDenseThreads, 1)
@@ -187,9 +195,16 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
   tc_fence_after();
   const int n_tiles = s_total;
   const int n_max = min(slot_capacity(p.E, p.S), kMaxSlots);
+  int ksplit = 1;
+  if (kMode == 2 && n_tiles > 0 && n_tiles < (int)gridDim.x) {
+    const int kb_min = (min(p.I, p.S > 0 ? p.Ish : p.I) + kBK - 1) / kBK;  // no part is empty
+    ksplit = max(1, min(min(kMaxKSplit, kb_min), (int)gridDim.x / n_tiles));
+  }
+  const int n_work = n_tiles * ksplit;  // work item w: K part w / n_tiles of tile w % n_tiles
   const uint32_t tmem_base = s_tmem;
-  auto tile_at = [&](int t) -> TileRef {
+  auto tile_at = [&](int w) -> TileRef {
     TileRef r;
+    const int t = w % n_tiles, part = w / n_tiles;
     r.j = find_item_slot(s_tab, n_max, t);
     const int4 sl = s_tab[r.j];
     r.kind = sl.x >> 16;
@@ -201,24 +216,23 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
     r.n0 = (local / mt) * kMaxBN;
     r.ntok = min(kMaxBN, r.T - r.n0);
     r.mext = kMode == 2 ? p.H : (r.kind ? p.Ish : p.I);
+    // contraction length: H for gate and up, the expert's I for down
+    const int kb = kMode == 2 ? ((r.kind ? p.Ish : p.I) + kBK - 1) / kBK : p.H / kBK;
+    r.kb0 = kb * part / ksplit;
+    r.kb1 = kb * (part + 1) / ksplit;
     return r;
-  };
-  // contraction length of a tile: H for gate and up, the expert's I for down
-  auto k_steps = [&](const TileRef& r) -> int {
-    return kMode == 2 ? ((r.kind ? p.Ish : p.I) + kBK - 1) / kBK : p.H / kBK;
   };
 
   if (warp == kProducerWarp) {
     if (lane == 0) {
       int it = 0;
-      for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x) {
+      for (int t = blockIdx.x; t < n_work && !*abort; t += gridDim.x) {
         const TileRef r = tile_at(t);
-        const int ks = k_steps(r);
         const int nb = (r.ntok + 31) / 32;  // 32-token boxes of B
         const CUtensorMap* ma = r.kind ? &maps.a_s : &maps.a_r;
         const int kb_rows = kMode == 2 ? r.expert * (r.kind ? p.Ish : p.I) : 0;
         const int a_row0 = kMode == 2 ? 0 : r.expert * r.mext + r.m0;
-        for (int k = 0; k < ks; ++k, ++it) {
+        for (int k = r.kb0; k < r.kb1; ++k, ++it) {
           const int s = it % kStages;
           if (!mbar_wait(&empty[s], ((it / kStages) & 1) ^ 1, abort, p.err)) break;
           unsigned char* sa = dsmem + s * kStageBytes;
@@ -243,9 +257,8 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
       int it = 0, tl = 0;
-      for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x, ++tl) {
+      for (int t = blockIdx.x; t < n_work && !*abort; t += gridDim.x, ++tl) {
         const TileRef r = tile_at(t);
-        const int ks = k_steps(r);
         const int nmma = (r.ntok + 15) & ~15;  // N of the instruction, a multiple of 16
         const uint32_t idesc = instr_desc(kMode == 2 ? 1 : 0, nmma);
         const int ab = tl & 1;
@@ -253,7 +266,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + ab * kMaxBN;
         bool ok = true;
-        for (int k = 0; k < ks; ++k, ++it) {
+        for (int k = r.kb0; k < r.kb1; ++k, ++it) {
           const int s = it % kStages;
           if (!mbar_wait(&full[s], (it / kStages) & 1, abort, p.err)) {
             ok = false;
@@ -269,7 +282,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
             const uint64_t ad = kMode == 2 ? smem_desc(a_addr + kk * 2048, kABytes / 2, 1024)
                                            : smem_desc(a_addr + kk * 32, 16, 1024);
             const uint64_t bd = smem_desc(b_addr + kk * 32, 16, 1024);
-            umma_bf16(d_tmem, ad, bd, idesc, (k > 0 || kk > 0) ? 1u : 0u);
+            umma_bf16(d_tmem, ad, bd, idesc, (k > r.kb0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&empty[s]);  // the stage is free once these MMAs have read it
         }
@@ -284,7 +297,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
     // ---------------- epilogue: warps 0-3, thread = one accumulator row (TMEM lane)
     int tl = 0;
     bool nan_seen = false;
-    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tl) {
+    for (int t = blockIdx.x; t < n_work; t += gridDim.x, ++tl) {
       // the four warps leave together (the named barriers below must never miss a warp)
       if (consumer_sync_or(128, *abort)) break;
       const TileRef r = tile_at(t);
