@@ -125,6 +125,19 @@ struct TileRef {
 // grid.  The gate and up GEMMs are never split: their epilogues are not linear in D.
 constexpr int kMaxKSplit = 4;
 
+// A gate or up launch with fewer tiles than CTAs (a large shared expert alone on this path:
+// I / 128 tiles) splits each slot's tokens into up to f N tiles, f = CTAs / tiles, at most
+// kMaxNSplit, each at least 16 tokens wide.  The CTAs of one M tile's N tiles run at the same
+// time, so the weights come from HBM once and from L2 for the others.  Every (neuron, token)
+// dot product keeps its K order, so the activations do not depend on the split.
+constexpr int kMaxNSplit = 8;
+
+// Token columns of one N tile of a slot with T tokens split f ways: a multiple of 16, at most
+// kMaxBN (f = 1: ceil(T / 256) tiles, 256 tokens wide but the last).
+__device__ __forceinline__ int ntile_width(int T, int f) {
+  return min(kMaxBN, ((T + f - 1) / f + 15) / 16 * 16);
+}
+
 template <int kMode>
 __global__ void __launch_bounds__(kDenseThreads, 1)
     dense_gemm_kernel(const __grid_constant__ DenseMaps maps, FwdParams p) {
@@ -165,6 +178,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
   pdl_trigger();
   pdl_wait();
   // tile table over the dense slots (every slot entry that can exist is read speculatively)
+  int nsplit = 1;  // N split of the gate and up GEMMs (kMaxNSplit)
   {
     const int n_slots = ld_cg(&p.meta[kMetaSlots]);
     const int n_max = min(slot_capacity(p.E, p.S), kMaxSlots);
@@ -183,6 +197,19 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
     }
     int total;
     int run = block_exclusive_scan(c, scratch, &total);
+    if (kMode != 2 && total > 0 && total < (int)gridDim.x) {
+      nsplit = min(kMaxNSplit, (int)gridDim.x / total);
+      if (nsplit > 1) {  // the same for every thread: recount the slots' tiles
+        c = 0;
+        for (int j = b0; j < b1; ++j) {
+          const int T = s_tab[j].y, w = ntile_width(T, nsplit);
+          const int v = s_tab[j].w ? s_mt[j] * ((T + w - 1) / w) : 0;
+          s_tab[j].w = v;
+          c += v;
+        }
+        run = block_exclusive_scan(c, scratch, &total);
+      }
+    }
     for (int j = b0; j < b1; ++j) {
       const int v = s_tab[j].w;
       s_tab[j].w = run;
@@ -211,10 +238,10 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
     r.expert = sl.x & 0xffff;
     r.T = sl.y;
     r.q0 = sl.z;
-    const int local = t - sl.w, mt = s_mt[r.j];
+    const int local = t - sl.w, mt = s_mt[r.j], wn = ntile_width(r.T, nsplit);
     r.m0 = (local % mt) * kBM;
-    r.n0 = (local / mt) * kMaxBN;
-    r.ntok = min(kMaxBN, r.T - r.n0);
+    r.n0 = (local / mt) * wn;
+    r.ntok = min(wn, r.T - r.n0);
     r.mext = kMode == 2 ? p.H : (r.kind ? p.Ish : p.I);
     // contraction length: H for gate and up, the expert's I for down
     const int kb = kMode == 2 ? ((r.kind ? p.Ish : p.I) + kBK - 1) / kBK : p.H / kBK;
