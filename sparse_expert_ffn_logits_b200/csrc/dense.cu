@@ -122,7 +122,7 @@ struct TileRef {
 // Largest K split of the down GEMM.  Its epilogue adds w * D into the output accumulator, so
 // partial sums over K ranges may be added separately.  A down GEMM with fewer tiles than CTAs
 // (a large shared expert alone on this path: H / 128 tiles) is split until its tiles cover the
-// grid.  The gate and up GEMMs are never split: their epilogues are not linear in D.
+// grid.  The gate and up GEMMs are never split over K: their epilogues are not linear in D.
 constexpr int kMaxKSplit = 4;
 
 // A gate or up launch with fewer tiles than CTAs (a large shared expert alone on this path:
