@@ -97,6 +97,23 @@ def test_forward_rejects_null_handle(lib):
     assert rc == moe.MOE_ERR_INVALID_ARG
 
 
+def test_other_entry_points_reject_null_handle(lib):
+    # every call that takes a handle checks it on the host, before any CUDA call
+    rw = moe.MoEExpertWeights(16, 16)
+    sp = moe.sparsity(("topk", 0.5))
+    p16 = ctypes.c_void_p(16)
+    for fn in (lib.moe_forward_host, lib.moe_forward_partial):
+        assert fn(None, p16, 1, p16, ctypes.byref(rw), None, ctypes.byref(sp), None, p16,
+                  None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_pack_experts(None, 0, p16, p16, p16, 1, p16, p16, None) == \
+        moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_profile_stages(None, None, 0) == moe.MOE_ERR_INVALID_ARG
+    buf = (ctypes.c_ulonglong * 4)()
+    assert lib.moe_read_trace(None, buf, 4) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_set_expert_range(None, 0, 1, 0) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_cast_output(None, p16, 1, p16, None) == moe.MOE_ERR_INVALID_ARG
+
+
 def test_status_strings(lib):
     for s in range(7):
         assert lib.moe_status_string(s)
