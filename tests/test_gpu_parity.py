@@ -154,6 +154,24 @@ def test_olmoe_full_batch(olmoe):
     _run(olmoe, 64, ("topk", 0.9), batch_index=8, expert_cache=cache)
 
 
+def test_olmoe_prefill_size_batch():
+    # the largest batch a handle takes (max_tokens = 1024): 128 tokens per expert on average, all
+    # on the tensor-core path.  Routing and kept sets of every token; the output of sampled
+    # tokens.
+    dl = DeviceLayer(synth.OLMOE, max_tokens=1024)
+    try:
+        # Allowance: five of the 8192 pairs swap a neuron across the cut.  The swaps are token 137
+        # pair 3 neuron 608, token 809 pair 4 neuron 491, token 240 pair 4 neuron 931, token 201
+        # pair 6 neuron 513, and token 120 pair 1 neuron 799.  Their oracle gaps are 3.7e-7 to
+        # 6.0e-7, against a band of 1e-6 * |cut|.  The fp32 bound of the 2048-term tensor-core
+        # gate is 7.6e-3 to 8.0e-3.
+        _run(dl, 1024, ("topk", 0.5), batch_index=11, tokens=np.arange(0, 1024, 33),
+             allow_fp32_bound=5)
+        assert moe_last_launches(dl.h) == 9
+    finally:
+        dl.close()
+
+
 def test_second_handle_keeps_first_working(olmoe):
     """A smaller handle created later must not shrink the kernels' shared-memory limits under
     the larger one that is still alive."""
